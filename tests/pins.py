@@ -1,0 +1,252 @@
+"""Checks that pin the float64 oracle to facts outside itself.
+
+Each check_* function raises AssertionError on failure.  test_oracle_pins.py runs
+them as tests; test_oracle_mutations.py plants plausible mistakes in the oracle
+(on the CPU) and confirms that at least one check catches each mistake.
+
+What pins what:
+* Hadamard: scipy.linalg.hadamard (textbook Sylvester routine), H H^T = d I in
+  integers, involution of H/sqrt(d), q.k preserved (blog section 2.1), Walsh
+  closed forms.
+* Codes: hand-written golden cases (tests/golden/bucket_cases.txt) for the strict
+  "<" chain of blog section 2.2.
+* Packing: hand-worked bytes (tests/golden/pack_cases.txt).
+* Distance: the |a-b| table (tests/golden/manhattan_table.txt), a pure-Python brute
+  force, and the t = 0 reduction to 3 x Hamming distance of sign bits (SimHash).
+* Top-k: pure-Python full sort by (distance, position); all-equal and k >= L cases.
+* Attention: budget = L equals torch's dense scaled-dot-product attention; budget 1
+  returns the V row.
+* GQA mapping and recall of planted keys on the seeded single-head workload.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle.adamas_ref as ref
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                rows.append(line.split())
+    return rows
+
+
+# ---------------------------------------------------------------- Hadamard
+def check_hadamard_matches_scipy():
+    import scipy.linalg
+    for n in (1, 2, 4, 8, 16, 32, 64, 128):
+        H = ref.sylvester_hadamard(n)
+        assert np.array_equal(H, scipy.linalg.hadamard(n).astype(np.int64)), n
+
+
+def check_hadamard_orthogonal():
+    H = ref.sylvester_hadamard(128)
+    assert np.array_equal(H @ H.T, 128 * np.eye(128, dtype=np.int64))
+
+
+def check_rotate_involution_and_dot():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((16, 128))
+    y = ref.hadamard_rotate(x)
+    assert np.allclose(ref.hadamard_rotate(y), x, rtol=0, atol=1e-12)
+    q, k = rng.standard_normal((2, 64, 128))
+    lhs = (ref.hadamard_rotate(q) * ref.hadamard_rotate(k)).sum(-1)
+    rhs = (q * k).sum(-1)
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+
+
+def check_rotate_closed_forms():
+    s = 1.0 / math.sqrt(128)
+    ones = np.ones(128)
+    e0 = np.zeros(128)
+    e0[0] = 1
+    assert np.allclose(ref.hadamard_rotate(ones), math.sqrt(128) * e0, atol=1e-12)
+    assert np.allclose(ref.hadamard_rotate(e0), s * ones, atol=1e-15)
+    # Walsh functions in natural order: e_1 -> + - + - ..., e_2 -> + + - - ...,
+    # e_64 -> 64 x (+) then 64 x (-)
+    e1 = np.zeros(128)
+    e1[1] = 1
+    assert np.allclose(ref.hadamard_rotate(e1), s * np.tile([1.0, -1.0], 64), atol=1e-15)
+    e2 = np.zeros(128)
+    e2[2] = 1
+    assert np.allclose(ref.hadamard_rotate(e2), s * np.tile([1.0, 1.0, -1.0, -1.0], 32),
+                       atol=1e-15)
+    e64 = np.zeros(128)
+    e64[64] = 1
+    assert np.allclose(ref.hadamard_rotate(e64),
+                       s * np.concatenate([np.ones(64), -np.ones(64)]), atol=1e-15)
+
+
+# ------------------------------------------------------------------- codes
+def check_bucket_golden():
+    for t, v, c in _golden("bucket_cases.txt"):
+        got = ref.bucketize(np.array([float(v)]), float(t))[0]
+        assert int(got) == int(c), (t, v, c, int(got))
+
+
+def check_pack_golden():
+    for row in _golden("pack_cases.txt"):
+        codes = np.array([int(x) for x in row[:4]], dtype=np.uint8)
+        byte = int(row[4])
+        assert int(ref.pack_codes(codes)[0]) == byte, (row, int(ref.pack_codes(codes)[0]))
+        assert np.array_equal(ref.unpack_codes(np.array([byte], np.uint8)), codes)
+    rng = np.random.default_rng(3)
+    c = rng.integers(0, 4, size=(5, 7, 128), dtype=np.uint8)
+    p = ref.pack_codes(c)
+    assert p.shape == (5, 7, 32)
+    assert np.array_equal(ref.unpack_codes(p), c)
+    # coordinate order across bytes: codes i % 4 -> every byte 0b11100100
+    assert np.all(ref.pack_codes(np.arange(128, dtype=np.uint8) % 4) == 228)
+
+
+# --------------------------------------------------------------- distances
+def check_manhattan_table():
+    table = np.array([[int(x) for x in r] for r in _golden("manhattan_table.txt")])
+    for a in range(4):
+        for b in range(4):
+            d = ref.manhattan(np.array([a]), np.array([[b]]))
+            assert int(d[0]) == table[a, b]
+
+
+def check_manhattan_bruteforce():
+    rng = np.random.default_rng(11)
+    for _ in range(5):
+        cq = rng.integers(0, 4, size=128)
+        ck = rng.integers(0, 4, size=(9, 128))
+        got = ref.manhattan(cq, ck)
+        for j in range(9):
+            s = 0
+            for i in range(128):
+                s += abs(int(cq[i]) - int(ck[j, i]))
+            assert got[j] == s
+    assert ref.manhattan(np.zeros(128, int), np.full((1, 128), 3))[0] == 384
+
+
+def check_simhash_reduction():
+    """t = 0: codes are 0/3 by sign, so distance = 3 x Hamming(sign bits)."""
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal(128)
+    K = rng.standard_normal((50, 128))
+    cq = ref.unpack_codes(ref.encode(q, 0.0))
+    ck = ref.unpack_codes(ref.encode(K, 0.0))
+    dist = ref.manhattan(cq, ck)
+    sq = ref.hadamard_rotate(q) >= 0
+    sk = ref.hadamard_rotate(K) >= 0
+    ham = (sq[None, :] != sk).sum(-1)
+    assert np.array_equal(dist, 3 * ham)
+
+
+# ------------------------------------------------------------------- top-k
+def check_topk_bruteforce():
+    rng = np.random.default_rng(13)
+    for L, k in ((1, 1), (5, 3), (37, 10), (100, 100), (100, 250), (300, 64)):
+        dist = rng.integers(0, 6, size=L)          # many ties
+        want = sorted(sorted(range(L), key=lambda j: (int(dist[j]), j))[:min(k, L)])
+        got = ref.select_topk(dist, k)
+        assert list(got) == want, (L, k)
+
+
+def check_topk_special():
+    assert list(ref.select_topk(np.full(50, 7), 8)) == list(range(8))
+    assert list(ref.select_topk(np.arange(10)[::-1].copy(), 20)) == list(range(10))
+    assert list(ref.select_topk(np.array([5, 1, 5, 0, 1]), 2)) == [1, 3]
+
+
+# --------------------------------------------------------------- attention
+def check_attention_dense():
+    rng = np.random.default_rng(17)
+    L = 200
+    q = rng.standard_normal(128)
+    K = rng.standard_normal((L, 128)) * 2
+    V = rng.standard_normal((L, 128))
+    got = ref.sparse_attention(q, K, V, np.arange(L))
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None, None, :], torch.from_numpy(K)[None, None],
+        torch.from_numpy(V)[None, None])[0, 0, 0].numpy()
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+    # a subset equals dense attention over just those rows
+    sub = np.array([3, 17, 50, 199])
+    want_sub = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None, None, :], torch.from_numpy(K[sub])[None, None],
+        torch.from_numpy(V[sub])[None, None])[0, 0, 0].numpy()
+    assert np.allclose(ref.sparse_attention(q, K, V, sub), want_sub, atol=1e-12)
+
+
+def check_attention_budget1():
+    rng = np.random.default_rng(19)
+    q = rng.standard_normal(128)
+    K = rng.standard_normal((10, 128))
+    V = rng.standard_normal((10, 128))
+    assert np.array_equal(ref.sparse_attention(q, K, V, np.array([4])), V[4])
+
+
+# -------------------------------------------------------------- whole step
+def check_decode_dense_limit():
+    """Budget = L: the sparse step is dense attention (v2 abstract's premise)."""
+    rng = np.random.default_rng(23)
+    B, Hq, Hkv, L = 2, 4, 2, 40
+    q = rng.standard_normal((B, Hq, 128))
+    K = rng.standard_normal((B, Hkv, L, 128))
+    V = rng.standard_normal((B, Hkv, L, 128))
+    idx, out = ref.decode_step(q, K, V, k=L, t=0.5)
+    assert np.array_equal(idx, np.broadcast_to(np.arange(L), (B, Hq, L)))
+    Kr = np.repeat(K, Hq // Hkv, axis=1)
+    Vr = np.repeat(V, Hq // Hkv, axis=1)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[:, :, None, :], torch.from_numpy(Kr),
+        torch.from_numpy(Vr))[:, :, 0].numpy()
+    assert np.allclose(out, want, atol=1e-12)
+
+
+def check_gqa_and_planted():
+    """Query head h reads kv head h // G: a copy of q_h planted only in that kv
+    head is its nearest key; the other kv heads never see it."""
+    rng = np.random.default_rng(29)
+    B, Hq, Hkv, L = 1, 8, 2, 256
+    G = Hq // Hkv
+    q = rng.standard_normal((B, Hq, 128))
+    K = rng.standard_normal((B, Hkv, L, 128))
+    V = rng.standard_normal((B, Hkv, L, 128))
+    pos = {}
+    for h in range(Hq):
+        p = 10 + 30 * h
+        K[0, h // G, p] = q[0, h]
+        pos[h] = p
+    idx, _ = ref.decode_step(q, K, V, k=1, t=0.5)
+    for h in range(Hq):
+        assert idx[0, h, 0] == pos[h], (h, idx[0, h, 0], pos[h])
+
+
+def check_planted_recall_single_head():
+    """Seeded single-head workload: its 4 planted keys (q + 0.1 noise) are in the
+    budget-64 selection."""
+    from workloads import WORKLOADS, generate
+    w = WORKLOADS[1]
+    inp = generate(w, "cpu")
+    q = inp.q.double().numpy()
+    K = inp.k_cache.double().numpy()
+    V = inp.v_cache.double().numpy()
+    idx, _ = ref.decode_step(q, K, V, k=64, t=inp.t)
+    planted = set(inp.planted[0, 0].tolist())
+    assert planted <= set(idx[0, 0].tolist())
+
+
+ALL_CHECKS = [
+    check_hadamard_matches_scipy, check_hadamard_orthogonal,
+    check_rotate_involution_and_dot, check_rotate_closed_forms, check_bucket_golden,
+    check_pack_golden, check_manhattan_table, check_manhattan_bruteforce,
+    check_simhash_reduction, check_topk_bruteforce, check_topk_special,
+    check_attention_dense, check_attention_budget1, check_decode_dense_limit,
+    check_gqa_and_planted, check_planted_recall_single_head,
+]

@@ -1,0 +1,135 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check the pins catch each.
+
+Every mutation replaces one oracle function for the duration of one test; at least
+one of the pin checks in tests/pins.py must then fail.
+"""
+import numpy as np
+import pytest
+
+import oracle.adamas_ref as ref
+from pins import ALL_CHECKS
+
+_orig = {name: getattr(ref, name) for name in (
+    "sylvester_hadamard", "hadamard_rotate", "bucketize", "pack_codes", "unpack_codes",
+    "manhattan", "select_topk", "sparse_attention", "decode_step")}
+
+
+def _h_or(n=128):                      # popcount(i | j) instead of i & j
+    idx = np.arange(n)
+    o = np.bitwise_or.outer(idx, idx)
+    par = np.zeros_like(o)
+    for b in range(int(n).bit_length()):
+        par ^= (o >> b) & 1
+    return np.where(par == 1, -1, 1).astype(np.int64)
+
+
+def _rotate_unscaled(x):               # forgot the 1/sqrt(d)
+    x = np.asarray(x, np.float64)
+    return x @ _orig["sylvester_hadamard"](x.shape[-1]).T.astype(np.float64)
+
+
+def _rotate_reversed(x):               # output coordinates in reversed order
+    return _orig["hadamard_rotate"](x)[..., ::-1]
+
+
+def _bucket_le(y, t):                  # "<=" instead of "<"
+    y = np.asarray(y, np.float64)
+    t = float(np.float32(t))
+    c = np.full(y.shape, 3, np.uint8)
+    c[y <= t] = 2
+    c[y <= 0] = 1
+    c[y <= -t] = 0
+    return c
+
+
+def _bucket_swapped(y, t):             # buckets 1 and 2 swapped
+    c = _orig["bucketize"](y, t)
+    out = c.copy()
+    out[c == 1] = 2
+    out[c == 2] = 1
+    return out
+
+
+def _pack_msb_first(codes):            # first coordinate in the top bits
+    c = np.asarray(codes, np.uint8)
+    c = c.reshape(c.shape[:-1] + (c.shape[-1] // 4, 4)).astype(np.uint16)
+    return (c[..., 3] | (c[..., 2] << 2) | (c[..., 1] << 4) | (c[..., 0] << 6)).astype(np.uint8)
+
+
+def _manhattan_sq(cq, ck):             # squared instead of absolute difference
+    a = np.asarray(cq, np.int64)
+    b = np.asarray(ck, np.int64)
+    return ((b - a[..., None, :]) ** 2).sum(-1)
+
+
+def _manhattan_dropped(cq, ck):        # dropped the last coordinate
+    a = np.asarray(cq, np.int64)[..., :-1]
+    b = np.asarray(ck, np.int64)[..., :-1]
+    return np.abs(b - a[..., None, :]).sum(-1)
+
+
+def _topk_high_pos(dist, k):           # ties go to the HIGHER position
+    dist = np.asarray(dist)
+    L = dist.shape[-1]
+    order = np.lexsort((-np.arange(L), dist))
+    return np.sort(order[:min(k, L)])
+
+
+def _topk_largest(dist, k):            # largest distance taken as most relevant
+    return _orig["select_topk"](-np.asarray(dist), k)
+
+
+def _attn_noscale(q, K, V, idx):       # forgot 1/sqrt(d)
+    q = np.asarray(q, np.float64)
+    s = np.asarray(K, np.float64)[idx] @ q
+    p = np.exp(s - s.max())
+    return (p / p.sum()) @ np.asarray(V, np.float64)[idx]
+
+
+def _attn_uses_k(q, K, V, idx):        # transposed operand: K rows used as values
+    return _orig["sparse_attention"](q, K, K, idx)
+
+
+def _decode_mod_gqa(q, K, V, k, t, key_codes=None, query_codes=None):
+    # query head h reads kv head h % Hkv instead of h // G
+    B, Hq, d = q.shape
+    Hkv = K.shape[1]
+    perm = [h % Hkv for h in range(Hq)]
+    G = Hq // Hkv
+    # reorder q so that the original routine's h // G lands on h % Hkv
+    inv = sorted(range(Hq), key=lambda h: (perm[h], h))
+    idx, out = _orig["decode_step"](q[:, inv], K, V, k, t)
+    back = np.argsort(inv)
+    return idx[:, back], out[:, back]
+
+
+MUTATIONS = {
+    "hadamard_or": ("sylvester_hadamard", _h_or),
+    "rotate_unscaled": ("hadamard_rotate", _rotate_unscaled),
+    "rotate_reversed": ("hadamard_rotate", _rotate_reversed),
+    "bucket_le": ("bucketize", _bucket_le),
+    "bucket_swapped": ("bucketize", _bucket_swapped),
+    "pack_msb_first": ("pack_codes", _pack_msb_first),
+    "manhattan_squared": ("manhattan", _manhattan_sq),
+    "manhattan_dropped_term": ("manhattan", _manhattan_dropped),
+    "topk_ties_high": ("select_topk", _topk_high_pos),
+    "topk_largest": ("select_topk", _topk_largest),
+    "attention_noscale": ("sparse_attention", _attn_noscale),
+    "attention_k_as_v": ("sparse_attention", _attn_uses_k),
+    "decode_gqa_modulo": ("decode_step", _decode_mod_gqa),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(ref, attr, fn)
+    failed = []
+    for check in ALL_CHECKS:
+        try:
+            check()
+        except AssertionError:
+            failed.append(check.__name__)
+        except Exception:               # a crash also counts as caught
+            failed.append(check.__name__ + "!")
+    assert failed, f"mutation {name} passed every pin"

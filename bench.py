@@ -1,0 +1,449 @@
+"""Benchmark of the Adamas decode step on B200: µs per step and effective HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--budget 128]
+                    [--impl ours|reference]
+
+Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32 query / 8 kv heads,
+d = 128, context 32768, bf16 K/V with 4 outlier channels, budget 128.  A "step" is
+one adamas_decode_step (query encode, distance scan, top-k, gather attention,
+combine: one cooperative kernel launch).
+
+Timing: inputs resident in HBM; R independent replicas of codes + K + V are
+rotated so the working set of consecutive steps exceeds 2x L2 (no cache reuse
+between steps); K steps are captured in CUDA graphs and timed with CUDA events on
+the launching stream, bracketed by barrier + synchronize; max over ranks.
+Multi-GPU: every rank runs its own replica set (weak scaling, no collective on the
+data path).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, generate, replicas_for_l2  # noqa: E402
+
+METRIC = "decode µs/step & effective HBM GB/s (% of roofline) at 32K ctx, budget 128"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "token_level_sparse_fwht_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload_key: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, or
+    None if there is none for this workload or the kernel source changed since."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(workload_key)
+    if not e or e.get("csrc_sha") != csrc_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms in the background."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- our arm
+def smi_id(dev) -> str:
+    """nvidia-smi id of a torch device (UUID, so CUDA_VISIBLE_DEVICES does not matter)."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index)
+
+
+def run_ours(args, rank, world, local):
+    import token_level_sparse_fwht_b200 as ad
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.config]
+    k = args.budget
+    L = w.L
+    t = w.t
+    # one "set" = everything one decode step touches: per layer (q, K, V, codes)
+    layer_sets = []
+    for layer in range(w.layers):
+        inp = generate(w, dev, layer=layer)
+        codes = torch.empty(inp.k_cache.shape[:-1] + (32,), dtype=torch.uint8, device=dev)
+        ad.encode_keys(inp.k_cache, codes, 0, L, t)
+        layer_sets.append((inp.q, inp.k_cache, inp.v_cache, codes))
+        del inp
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    append = w.append
+    step_bytes = w.algorithmic_bytes(k) * w.layers
+    if append:
+        step_bytes += w.B * w.Hkv * append * (128 * w.elem_bytes + 32)
+    R = args.replicas or replicas_for_l2(step_bytes, l2, 2.0)
+    sets = [layer_sets]
+    for _ in range(R - 1):
+        sets.append([tuple(x.clone() for x in ls) for ls in layer_sets])
+    ws = ad.decode_workspace(w.B, w.Hq, w.Hkv, L, k, dev)
+    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    plan = ad.decode_plan(w.B, w.Hq, w.Hkv, L, k)
+    launches_per_step = w.layers * (2 if append else 1)
+
+    def step(i, s, q_override=None):
+        for (q, kc, vc, cd) in sets[i % R]:
+            if append:
+                ad.encode_keys(kc, cd, L - append, append, t, stream=s)
+            ad.decode_step(q if q_override is None else q_override, kc, vc, cd, L, k, t, ws,
+                           out=out, stream=s)
+
+    # eager warm-up (also loads the kernels and sets their attributes)
+    with torch.cuda.stream(stream):
+        for i in range(max(3, min(args.warmup, 3 * R))):
+            step(i, stream)
+    stream.synchronize()
+    ad.check_workspace(ws, stream)
+
+    # CUDA graphs of `chunk` steps (rotating replicas) + one for the remainder
+    K = args.steps
+    chunk = max(1, min(K, 1000 // launches_per_step))
+    graphs = []
+    use_graph = True
+    try:
+        sizes = ([chunk] if K >= chunk else []) + ([K % chunk] if K % chunk else [])
+        for n in sizes:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(n):
+                        step(i, stream)
+            graphs.append((n, g))
+    except Exception as e:  # capture unsupported: launch eagerly
+        use_graph = False
+        graphs = []
+        print(f"# graph capture failed ({e}); eager launches", file=sys.stderr)
+    stream.synchronize()
+
+    def timed_region():
+        if use_graph:
+            for _ in range(K // chunk):
+                graphs[0][1].replay()
+            if K % chunk:
+                graphs[-1][1].replay()
+        else:
+            for i in range(K):
+                step(i, stream)
+
+    with torch.cuda.stream(stream):       # graph warm-up replays
+        for _ in range(max(1, args.warmup // max(1, chunk))):
+            if use_graph:
+                graphs[0][1].replay()
+            else:
+                step(0, stream)
+    stream.synchronize()
+
+    sampler = ClockSampler(smi_id(dev))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        timed_region()
+        e1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    ad.check_workspace(ws, stream)
+    del graphs
+
+    # e2e through the public API with host buffers: every step copies its queries in
+    # from pinned host memory and reads the fp32 output back
+    q_host = torch.stack([ls[0] for ls in layer_sets]).cpu().pin_memory()
+    out_host = torch.empty((w.layers,) + tuple(out.shape), dtype=torch.float32).pin_memory()
+    q_dev = torch.empty(q_host.shape, dtype=q_host.dtype, device=dev)
+    outs = torch.empty(out_host.shape, dtype=torch.float32, device=dev)
+    K2 = max(3, min(K, 2000 // w.layers))
+
+    def e2e_step(i):
+        q_dev.copy_(q_host, non_blocking=True)
+        for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
+            if append:
+                ad.encode_keys(kc, cd, L - append, append, t, stream=stream)
+            ad.decode_step(q_dev[li], kc, vc, cd, L, k, t, ws, out=outs[li], stream=stream)
+        out_host.copy_(outs, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            e2e_step(i)
+    stream.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for i in range(K2):
+            e2e_step(i)
+        f1.record(stream)
+    stream.synchronize()
+    ms_e2e = f0.elapsed_time(f1)
+
+    # max over ranks
+    tt = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+    ms, ms_e2e = float(tt[0]), float(tt[1])
+    return dict(w=w, k=k, ms=ms, ms_e2e=ms_e2e, K=K, K2=K2, R=R, step_bytes=step_bytes,
+                clocks=clocks, plan=plan, use_graph=use_graph,
+                launches=K * launches_per_step,
+                h2d=q_host.numel() * q_host.element_size(),
+                d2h=out_host.numel() * out_host.element_size())
+
+
+# --------------------------------------------------- float64 oracle on host
+def oracle_inputs(w, seed_device="cpu"):
+    import numpy as np  # noqa: F401
+    import oracle
+    inp = generate(w, seed_device)
+    q = inp.q.double().cpu().numpy()
+    K = inp.k_cache.double().cpu().numpy()
+    V = inp.v_cache.double().cpu().numpy()
+    return inp.t, q, K, V, oracle
+
+
+def cpu_baseline(w, k, budget_s=12.0):
+    """The oracle's full decode step (all heads) on the host, repeated for about
+    budget_s seconds: effective GB/s over the same algorithmic bytes."""
+    t, q, K, V, oracle = oracle_inputs(w)
+    kc = oracle.encode(K, t)        # key codes are cache state, built before timing
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.decode_step(q, K, V, k, t, key_codes=kc)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 50:
+            break
+    per_step = el / n
+    return {"value": w.algorithmic_bytes(k) / per_step / 1e9, "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{n} full decode steps of the same workload (all {w.B * w.Hq} heads), "
+                      f"{per_step * 1e3:.0f} ms each, numpy float64, single thread"}
+
+
+def run_reference(args):
+    """--impl reference: the float64 oracle as the reference arm.  Each of the K steps
+    is one query head over a contiguous key slice sized so the whole run takes about
+    a minute; GB/s is computed over the sample's own algorithmic bytes."""
+    w = WORKLOADS[args.config]
+    k = args.budget
+    t, q, K, V, oracle = oracle_inputs(w)
+    G = w.G
+    nsteps = args.steps + args.warmup
+    # calibrate: seconds per key of one head's decode
+    S0 = min(w.L, 4096)
+    kc0 = oracle.encode(K[0, 0, :S0], t)
+    t0 = time.perf_counter()
+    oracle.decode_head(q[0, 0], K[0, 0, :S0], V[0, 0, :S0], k, t, key_codes_rows=kc0)
+    per_key = (time.perf_counter() - t0) / S0
+    S = int(max(256, min(w.L, 60.0 / max(1, nsteps) / per_key)))
+    kcs = {}
+    tot = 0.0
+    nbytes = 0
+    for i in range(nsteps):
+        h = i % w.Hq
+        kv = h // G
+        lo = (i * 7919) % max(1, w.L - S + 1)
+        key = (kv, lo)
+        if key not in kcs:
+            kcs[key] = oracle.encode(K[0, kv, lo:lo + S], t)
+        a = time.perf_counter()
+        oracle.decode_head(q[0, h], K[0, kv, lo:lo + S], V[0, kv, lo:lo + S], k, t,
+                           key_codes_rows=kcs[key])
+        b = time.perf_counter()
+        if i >= args.warmup:
+            tot += b - a
+            nbytes += S * 32 + min(k, S) * 2 * 128 * w.elem_bytes + 128 * (w.elem_bytes + 4)
+        if len(kcs) > 64:
+            kcs.clear()
+    gbs = nbytes / tot / 1e9
+    return {
+        "metric": METRIC, "value": round(gbs, 6), "unit": "GB/s", "impl": "reference",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot / max(1, args.steps) * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128, "L": w.L,
+                   "k": k, "sample_keys_per_step": S},
+        "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: one query head over {S} consecutive keys "
+                                   f"(budget min({k}, {S})), numpy float64, single thread"},
+        "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(WORKLOADS))
+    ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--replicas", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.budget is None:
+        args.budget = 128 if 128 in WORKLOADS[args.config].budgets else WORKLOADS[args.config].budgets[0]
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    r = run_ours(args, rank, world, local)
+    w, k = r["w"], r["k"]
+    peak, peak_kind = peaks()
+    per_step_s = r["ms"] / 1e3 / r["K"]
+    gbs_rank = r["step_bytes"] / per_step_s / 1e9
+    value = gbs_rank * world
+    e2e_step_s = r["ms_e2e"] / 1e3 / r["K2"]
+    key = f"config{args.config}_k{k}"
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": r["K"],
+        "warmup": args.warmup,
+        "ms_per_step": round(r["ms"] / r["K"], 6),
+        "us_per_step": round(per_step_s * 1e6, 3),
+        "pct_of_roofline": round(100 * gbs_rank / peak, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u8-codes/bf16-kv/f32-acc" if w.elem_bytes == 2 else "u8-codes/f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128, "L": w.L,
+                   "k": k, "algorithmic_bytes_per_step": r["step_bytes"],
+                   "replicas": r["R"], "l2": "rotated replicas, working set >= 2x L2",
+                   "layers": w.layers, "append_tokens": w.append,
+                   "graph": r["use_graph"], "ctas": r["plan"]["ctas"],
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(gbs_rank / peak, 4),
+                     "traffic": ncu_traffic(key),
+                     "kernel": "decode_kernel (one launch per step)",
+                     "peak_source": f"{peak_kind} hbm_gbs"},
+        "e2e": {"value": round(r["step_bytes"] * world / e2e_step_s / 1e9, 2), "unit": "GB/s",
+                "us_per_step": round(e2e_step_s * 1e6, 3),
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, k)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

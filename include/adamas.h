@@ -1,0 +1,157 @@
+/*
+ * adamas.h — C ABI of the Adamas decode hot path on B200 (sm_100a).
+ *
+ * The method ("Adamas: Hadamard Sparse Attention for Efficient Long-Context
+ * Inference", arXiv 2510.18413, v2 abstract): every key and every decode query is
+ * passed through a Hadamard transform, bucketized and compressed to 2-bit codes; a
+ * distance between the query code and every key code (a Manhattan distance, per
+ * the v1 abstract) picks the top-k candidate positions; the ORIGINAL K/V rows at
+ * those positions are gathered for exact sparse attention.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers, owned by the caller.  The library
+ *    never allocates, frees or synchronizes in these calls (except
+ *    adamas_check_workspace, which says so), and keeps no per-call host state.
+ *  - Every call is asynchronous on `stream`; argument checks run on the host
+ *    before any launch, and a rejected call launches nothing.
+ *  - Layouts are contiguous, row-major:
+ *        q        [B][Hq][d]           elements of `dt`
+ *        k_cache  [B][Hkv][Lmax][d]    elements of `dt`   (original keys)
+ *        v_cache  [B][Hkv][Lmax][d]    elements of `dt`
+ *        codes    [B][Hkv][Lmax][d/4]  bytes: 2-bit codes, 4 per byte, coordinate
+ *                                      i in byte i>>2 at bits 2*(i&3)
+ *        qcodes   [B][Hq][d/4]         bytes, same packing
+ *        idx      [B][Hq][k_eff]       int32 positions, ascending
+ *        out      [B][Hq][d]           float32
+ *    with d = 128, G = Hq / Hkv query heads per kv head (query head h reads kv
+ *    head h / G), and k_eff = min(k, L).
+ *  - Pointers must be 16-byte aligned (idx: 4-byte, workspace: 256-byte).
+ *  - Codes: y = H x / sqrt(d) with H the natural-order Sylvester Hadamard matrix,
+ *    then code = [y >= -t] + [y >= 0] + [y >= t] in {0,1,2,3} (the blog section 2.2
+ *    rule of three thresholds compared with strict "<", here at {-t, 0, +t} with a
+ *    fixed per-run t >= 0 shared by keys and queries).
+ *  - Selection: query head h keeps the k_eff positions with the smallest
+ *    Manhattan distance between its code and the key codes of kv head h / G, ties
+ *    going to the lower position.
+ *  - Attention: softmax over the selected positions of (q . K_j) / sqrt(d), fp32
+ *    accumulation, fp32 output.
+ *
+ * Errors: ADAMAS_ERR_INVALID_ARG for null or misaligned pointers, non-positive
+ * sizes, L > Lmax, Hq % Hkv != 0, t < 0 or not finite, a too-small workspace;
+ * ADAMAS_ERR_UNSUPPORTED for d != 128, G not in {1, 2, 4, 8}, or a context too long
+ * for the on-chip plan; ADAMAS_ERR_CUDA when a launch fails (no C++ exception ever
+ * crosses this boundary).
+ */
+#ifndef ADAMAS_H
+#define ADAMAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ADAMAS_OK = 0,
+  ADAMAS_ERR_INVALID_ARG = 1,
+  ADAMAS_ERR_UNSUPPORTED = 2,
+  ADAMAS_ERR_CUDA = 3,
+  ADAMAS_ERR_TIMEOUT = 4
+} adamas_status;
+
+typedef enum { ADAMAS_F32 = 0, ADAMAS_BF16 = 1 } adamas_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* adamas_status_string(adamas_status s);
+
+/* ABI version, bumped when a signature or layout changes. */
+int adamas_abi_version(void);
+
+/*
+ * Key encoder, run when keys are appended to the cache (v2 abstract: Hadamard
+ * transform, bucketization, 2-bit compression of the keys).  Encodes positions
+ * [pos0, pos0 + n_new) of every (batch, kv head) from k_cache into codes.
+ * Reads n_new * B * Hkv * d elements, writes n_new * B * Hkv * d/4 bytes.
+ */
+adamas_status adamas_encode_keys(const void* k_cache, adamas_dtype dt, int B, int Hkv, int d,
+                                 int64_t Lmax, int64_t pos0, int64_t n_new, float t,
+                                 uint8_t* codes, cudaStream_t stream);
+
+/* Query encoder: the same transform on q [B][Hq][d] into qcodes [B][Hq][d/4]. */
+adamas_status adamas_encode_queries(const void* q, adamas_dtype dt, int B, int Hq, int d,
+                                    float t, uint8_t* qcodes, cudaStream_t stream);
+
+/*
+ * Workspace of adamas_decode_step and adamas_select_topk, in bytes; 0 if the
+ * arguments are invalid or unsupported.  The decode kernel keeps all its
+ * intermediate data on chip, so the workspace only holds the device error word
+ * that a bounded wait sets when it gives up (see adamas_check_workspace).  Zero-fill
+ * it once before first use (adamas_workspace_init); any number of calls, on any
+ * stream, may share it.
+ */
+size_t adamas_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k);
+
+/* Zero-fills a workspace (cudaMemsetAsync on `stream`). */
+adamas_status adamas_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * SYNCHRONIZES `stream`, then reads the device error word of a decode workspace.
+ * Returns ADAMAS_ERR_TIMEOUT if a kernel gave up a bounded wait (completion of a
+ * bulk copy into shared memory) since the workspace was initialised, else
+ * ADAMAS_OK (or ADAMAS_ERR_CUDA if the stream reported an error).
+ */
+adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * One decode step, all five stages in ONE kernel launch (thread-block clusters,
+ * one cluster per (batch, kv head) pair, cross-CTA exchange in distributed shared
+ * memory): query encode, distance scan over the key codes, exact per-head top-k,
+ * gather of the original K/V rows with split softmax attention, and the combine of
+ * the splits.
+ * Uses the first L positions of every cache row; codes must hold the keys' codes
+ * for those positions (adamas_encode_keys).  idx_out may be NULL; when given it
+ * receives the selected positions [B][Hq][k_eff], ascending.
+ */
+adamas_status adamas_decode_step(const void* q, const void* k_cache, const void* v_cache,
+                                 const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                 int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
+                                 void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                 float* out, cudaStream_t stream);
+
+/*
+ * Stage entry point: distance scan + top-k from given query codes (no attention).
+ * Same kernel as adamas_decode_step with the attention stages switched off.
+ */
+adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, int B, int Hq,
+                                 int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
+                                 size_t ws_bytes, int32_t* idx_out, cudaStream_t stream);
+
+/* Workspace of adamas_sparse_attention, in bytes (zero-filled once, self-cleaning). */
+size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff);
+
+/*
+ * Stage entry point: split-k gather attention + combine over explicit positions
+ * idx [B][Hq][k_eff] (any order, each in [0, Lmax)); writes out [B][Hq][d] fp32.
+ */
+adamas_status adamas_sparse_attention(const void* q, const void* k_cache, const void* v_cache,
+                                      adamas_dtype dt, const int32_t* idx, int B, int Hq,
+                                      int Hkv, int d, int64_t Lmax, int k_eff, void* workspace,
+                                      size_t ws_bytes, float* out, cudaStream_t stream);
+
+/*
+ * Launch plan of adamas_decode_step for these sizes on the current device (host
+ * only, no launch): total CTAs, CTAs per thread-block cluster (one cluster per
+ * (batch, kv head) pair), key positions per CTA, dynamic shared memory bytes per
+ * CTA.  Any output pointer may be NULL.
+ */
+adamas_status adamas_decode_plan(int B, int Hq, int Hkv, int d, int64_t L, int k, int* ctas,
+                                 int* cluster, int64_t* tokens_per_cta, int* smem_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ADAMAS_H */

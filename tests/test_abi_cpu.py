@@ -1,0 +1,114 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry point
+declared in include/adamas.h, and rejects bad arguments on the host before any
+launch (none of these calls reaches a kernel)."""
+import math
+
+import pytest
+
+import token_level_sparse_fwht_b200 as ad
+from token_level_sparse_fwht_b200 import (OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, F32, BF16)
+
+A = 1 << 20          # a fake, 256-byte aligned "device" address; never dereferenced
+MIS = A + 1          # misaligned
+
+
+def test_library_exports_every_header_symbol():
+    lib = ad.lib()
+    syms = ad.header_symbols()
+    assert "adamas_decode_step" in syms and "adamas_encode_keys" in syms
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert lib.adamas_abi_version() == 1
+
+
+def test_status_strings():
+    assert ad.status_string(OK) == "ok"
+    assert "invalid" in ad.status_string(ERR_INVALID_ARG)
+    assert ad.status_string(99) == "unknown status"
+
+
+def _decode(**kw):
+    a = dict(q=A, kc=A, v=A, codes=A, dt=BF16, B=1, Hq=32, Hkv=8, d=128, Lmax=4096, L=4096, k=128,
+             t=1.0, ws=A, ws_bytes=0, idx=None, out=A, stream=None)
+    a.update(kw)
+    return ad.lib().adamas_decode_step(a["q"], a["kc"], a["v"], a["codes"], a["dt"], a["B"],
+                                       a["Hq"], a["Hkv"], a["d"], a["Lmax"], a["L"], a["k"],
+                                       a["t"], a["ws"], a["ws_bytes"], a["idx"], a["out"],
+                                       a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), ERR_INVALID_ARG),
+    (dict(out=None), ERR_INVALID_ARG),
+    (dict(ws=None), ERR_INVALID_ARG),
+    (dict(d=64), ERR_UNSUPPORTED),
+    (dict(Hq=24, Hkv=8), ERR_UNSUPPORTED),       # G = 3
+    (dict(Hq=30, Hkv=8), ERR_INVALID_ARG),       # Hq % Hkv != 0
+    (dict(L=5000), ERR_INVALID_ARG),             # L > Lmax
+    (dict(L=0), ERR_INVALID_ARG),
+    (dict(k=0), ERR_INVALID_ARG),
+    (dict(B=0), ERR_INVALID_ARG),
+    (dict(t=-0.5), ERR_INVALID_ARG),
+    (dict(t=math.nan), ERR_INVALID_ARG),
+    (dict(t=math.inf), ERR_INVALID_ARG),
+    (dict(dt=7), ERR_INVALID_ARG),
+    (dict(q=MIS), ERR_INVALID_ARG),
+    (dict(codes=A + 8), ERR_INVALID_ARG),
+    (dict(ws=A + 16), ERR_INVALID_ARG),          # workspace needs 256-byte alignment
+    (dict(idx=A + 2), ERR_INVALID_ARG),
+    (dict(ws_bytes=128), ERR_INVALID_ARG),       # too small (needs 256)
+])
+def test_decode_rejects_before_launch(kw, status):
+    assert _decode(**kw) == status
+
+
+def test_encode_keys_rejects():
+    f = ad.lib().adamas_encode_keys
+    assert f(None, BF16, 1, 8, 128, 100, 0, 10, 1.0, A, None) == ERR_INVALID_ARG
+    assert f(A, BF16, 1, 8, 128, 100, 95, 10, 1.0, A, None) == ERR_INVALID_ARG   # past Lmax
+    assert f(A, BF16, 1, 8, 128, 100, -1, 10, 1.0, A, None) == ERR_INVALID_ARG
+    assert f(A, BF16, 1, 8, 128, 100, 0, 0, 1.0, A, None) == ERR_INVALID_ARG
+    assert f(A, BF16, 1, 8, 96, 100, 0, 10, 1.0, A, None) == ERR_UNSUPPORTED
+    assert f(A, F32, 1, 8, 128, 100, 0, 10, -1.0, A, None) == ERR_INVALID_ARG
+    assert f(MIS, F32, 1, 8, 128, 100, 0, 10, 1.0, A, None) == ERR_INVALID_ARG
+    g = ad.lib().adamas_encode_queries
+    assert g(A, BF16, 1, 32, 128, 1.0, None, None) == ERR_INVALID_ARG
+    assert g(A, BF16, 0, 32, 128, 1.0, A, None) == ERR_INVALID_ARG
+
+
+def test_select_and_attention_reject():
+    s = ad.lib().adamas_select_topk
+    assert s(None, A, 1, 32, 8, 100, 100, 10, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    assert s(A, A, 1, 32, 8, 100, 100, 10, A, 1 << 30, None, None) == ERR_INVALID_ARG
+    assert s(A, A, 1, 32, 8, 100, 101, 10, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    assert s(A, A, 1, 48, 8, 100, 100, 10, A, 1 << 30, A, None) == ERR_UNSUPPORTED
+    assert s(A, A, 1, 32, 8, 100, 100, 10, A, 16, A, None) == ERR_INVALID_ARG
+    at = ad.lib().adamas_sparse_attention
+    assert at(A, A, A, BF16, None, 1, 32, 8, 128, 100, 10, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    assert at(A, A, A, BF16, A, 1, 32, 8, 64, 100, 10, A, 1 << 30, A, None) == ERR_UNSUPPORTED
+    assert at(A, A, A, BF16, A, 1, 32, 8, 128, 100, 10, A, 8, A, None) == ERR_INVALID_ARG
+    assert at(A, A, A, BF16, A + 1, 1, 32, 8, 128, 100, 10, A, 1 << 30, A, None) == ERR_INVALID_ARG
+
+
+def test_workspace_sizes_and_plan():
+    n = ad.decode_workspace_bytes(1, 32, 8, 32768, 128)
+    assert n > 0 and n % 256 == 0
+    assert ad.lib().adamas_decode_workspace_bytes(1, 32, 8, 64, 32768, 128) == 0
+    assert ad.lib().adamas_decode_workspace_bytes(1, 32, 8, 128, 0, 128) == 0
+    assert ad.lib().adamas_sparse_attention_workspace_bytes(1, 32, 128) > 0
+    assert ad.lib().adamas_sparse_attention_workspace_bytes(1, 32, 0) == 0
+    # without a device the plan assumes a 148-SM B200 and its shared-memory cap
+    p = ad.decode_plan(1, 32, 8, 32768, 128)           # 8 units: clusters of 16
+    assert p == {"ctas": 128, "cluster": 16, "tokens_per_cta": 2048,
+                 "smem_bytes": p["smem_bytes"]} and p["smem_bytes"] <= 232448
+    big = ad.decode_plan(8, 32, 8, 32768, 1024)         # 64 units: clusters of 2
+    assert big["cluster"] == 2 and big["tokens_per_cta"] == 16384
+    for args in [(4, 32, 8, 131072, 1024), (1, 32, 32, 131072, 1024), (1, 2, 1, 70000, 50),
+                 (75, 4, 4, 64, 8), (1, 1, 1, 1024, 64)]:
+        q = ad.decode_plan(*args)
+        B, Hq, Hkv, L, k = args
+        assert q["ctas"] == B * Hkv * q["cluster"] and 1 <= q["cluster"] <= 16
+        assert q["tokens_per_cta"] * q["cluster"] >= L and q["tokens_per_cta"] <= 65535
+        assert q["smem_bytes"] <= 232448
+    tiny = ad.decode_plan(3, 4, 4, 1, 1)                # L = 1: one key per unit
+    assert tiny["cluster"] == 1 and tiny["tokens_per_cta"] == 1 and tiny["ctas"] == 12

@@ -1,0 +1,237 @@
+"""Adamas decode hot path on B200: thin Python binding of libadamas.so.
+
+Every step of the path runs in the library's CUDA kernels; this module only
+marshals torch tensors (device memory, streams) into the C ABI declared in
+include/adamas.h.  There is no CPU fallback: if the library is missing or a call
+fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libadamas.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "adamas.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
+F32, BF16 = 0, 1
+HEAD_DIM = 128
+
+
+class AdamasError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+_c_i = ctypes.c_int
+_c_i64 = ctypes.c_int64
+_c_f = ctypes.c_float
+_c_sz = ctypes.c_size_t
+_c_p = ctypes.c_void_p
+
+_SIGNATURES = {
+    "adamas_status_string": (ctypes.c_char_p, [_c_i]),
+    "adamas_abi_version": (_c_i, []),
+    "adamas_encode_keys": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i64, _c_f,
+                                  _c_p, _c_p]),
+    "adamas_encode_queries": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p]),
+    "adamas_decode_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i64, _c_i]),
+    "adamas_workspace_init": (_c_i, [_c_p, _c_sz, _c_p]),
+    "adamas_check_workspace": (_c_i, [_c_p, _c_sz, _c_p]),
+    "adamas_decode_step": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i64,
+                                  _c_i64, _c_i, _c_f, _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "adamas_select_topk": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i, _c_p,
+                                  _c_sz, _c_p, _c_p]),
+    "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
+    "adamas_sparse_attention": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i, _c_i,
+                                       _c_i64, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "adamas_decode_plan": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i64, _c_i,
+                                  ctypes.POINTER(_c_i), ctypes.POINTER(_c_i),
+                                  ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i)]),
+}
+
+
+def lib():
+    """The loaded libadamas.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m token_level_sparse_fwht_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_symbols():
+    """Entry points declared in include/adamas.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(adamas_[a-z_0-9]+)\s*\(", text)))
+
+
+def status_string(s: int) -> str:
+    return lib().adamas_status_string(int(s)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise AdamasError(status, what)
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+# ------------------------------------------------------------------ encoders
+def encode_keys(k_cache: torch.Tensor, codes: torch.Tensor, pos0: int, n_new: int, t: float,
+                stream=None):
+    """Encodes positions [pos0, pos0+n_new) of k_cache [B,Hkv,Lmax,128] into codes
+    [B,Hkv,Lmax,32] (uint8)."""
+    B, Hkv, Lmax, d = k_cache.shape
+    if codes.dtype != torch.uint8 or tuple(codes.shape) != (B, Hkv, Lmax, d // 4):
+        raise ValueError("codes must be uint8 [B, Hkv, Lmax, d/4]")
+    _check(lib().adamas_encode_keys(_dev(k_cache, "k_cache"), _dtype_code(k_cache), B, Hkv, d,
+                                    Lmax, pos0, n_new, float(t), _dev(codes, "codes"),
+                                    _stream(stream)), "adamas_encode_keys")
+    return codes
+
+
+def encode_queries(q: torch.Tensor, t: float, qcodes: torch.Tensor | None = None, stream=None):
+    B, Hq, d = q.shape
+    if qcodes is None:
+        qcodes = torch.empty((B, Hq, d // 4), dtype=torch.uint8, device=q.device)
+    _check(lib().adamas_encode_queries(_dev(q, "q"), _dtype_code(q), B, Hq, d, float(t),
+                                       _dev(qcodes, "qcodes"), _stream(stream)),
+           "adamas_encode_queries")
+    return qcodes
+
+
+# ---------------------------------------------------------------- workspace
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, L: int, k: int) -> int:
+    n = lib().adamas_decode_workspace_bytes(B, Hq, Hkv, HEAD_DIM, L, k)
+    if n == 0:
+        raise AdamasError(ERR_INVALID_ARG, "adamas_decode_workspace_bytes")
+    return int(n)
+
+
+def decode_plan(B: int, Hq: int, Hkv: int, L: int, k: int) -> dict:
+    ctas, cluster, smem = _c_i(), _c_i(), _c_i()
+    rng = _c_i64()
+    _check(lib().adamas_decode_plan(B, Hq, Hkv, HEAD_DIM, L, k, ctypes.byref(ctas),
+                                    ctypes.byref(cluster), ctypes.byref(rng),
+                                    ctypes.byref(smem)), "adamas_decode_plan")
+    return {"ctas": ctas.value, "cluster": cluster.value, "tokens_per_cta": rng.value,
+            "smem_bytes": smem.value}
+
+
+def init_workspace(ws: torch.Tensor, stream=None):
+    _check(lib().adamas_workspace_init(_dev(ws, "workspace"), ws.numel(), _stream(stream)),
+           "adamas_workspace_init")
+    return ws
+
+
+def decode_workspace(B: int, Hq: int, Hkv: int, L: int, k: int, device="cuda", stream=None):
+    """A zero-initialised decode workspace (torch allocates, the library zero-fills)."""
+    n = decode_workspace_bytes(B, Hq, Hkv, L, k)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    return init_workspace(ws, stream)
+
+
+def check_workspace(ws: torch.Tensor, stream=None):
+    """Synchronizes the stream; raises AdamasError(ERR_TIMEOUT) if a device wait gave up."""
+    _check(lib().adamas_check_workspace(_dev(ws, "workspace"), ws.numel(), _stream(stream)),
+           "adamas_check_workspace")
+
+
+# -------------------------------------------------------------- decode step
+def decode_step(q, k_cache, v_cache, codes, L: int, k: int, t: float, ws, idx_out=None,
+                out=None, stream=None):
+    """One decode step (fused kernel).  Returns out [B,Hq,128] fp32 (and fills idx_out
+    [B,Hq,min(k,L)] int32 if given)."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
+    _check(lib().adamas_decode_step(_dev(q, "q"), _dev(k_cache, "k_cache"),
+                                    _dev(v_cache, "v_cache"), _dev(codes, "codes"),
+                                    _dtype_code(k_cache), B, Hq, Hkv, d, Lmax, L, k, float(t),
+                                    _dev(ws, "workspace"), ws.numel(), idx_ptr,
+                                    _dev(out, "out"), _stream(stream)), "adamas_decode_step")
+    return out
+
+
+def select_topk(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
+    B, Hq, _ = qcodes.shape
+    _, Hkv, Lmax, _ = codes.shape
+    k_eff = min(k, L)
+    if idx_out is None:
+        idx_out = torch.empty((B, Hq, k_eff), dtype=torch.int32, device=qcodes.device)
+    _check(lib().adamas_select_topk(_dev(qcodes, "qcodes"), _dev(codes, "codes"), B, Hq, Hkv,
+                                    Lmax, L, k, _dev(ws, "workspace"), ws.numel(),
+                                    _dev(idx_out, "idx_out"), _stream(stream)),
+           "adamas_select_topk")
+    return idx_out
+
+
+def sparse_attention_workspace(B: int, Hq: int, k_eff: int, device="cuda", stream=None):
+    n = int(lib().adamas_sparse_attention_workspace_bytes(B, Hq, k_eff))
+    if n == 0:
+        raise AdamasError(ERR_INVALID_ARG, "adamas_sparse_attention_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    return init_workspace(ws, stream)
+
+
+def sparse_attention(q, k_cache, v_cache, idx, ws=None, out=None, stream=None):
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    k_eff = idx.shape[-1]
+    if idx.dtype != torch.int32:
+        raise TypeError("idx must be int32")
+    if ws is None:
+        ws = sparse_attention_workspace(B, Hq, k_eff, q.device, stream)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _check(lib().adamas_sparse_attention(_dev(q, "q"), _dev(k_cache, "k_cache"),
+                                         _dev(v_cache, "v_cache"), _dtype_code(k_cache),
+                                         _dev(idx, "idx"), B, Hq, Hkv, d, Lmax, k_eff,
+                                         _dev(ws, "workspace"), ws.numel(), _dev(out, "out"),
+                                         _stream(stream)), "adamas_sparse_attention")
+    return out
+
+
+__all__ = ["lib", "header_symbols", "status_string", "AdamasError", "encode_keys",
+           "encode_queries", "decode_workspace_bytes", "decode_plan", "init_workspace",
+           "decode_workspace", "check_workspace", "decode_step", "select_topk",
+           "sparse_attention_workspace", "sparse_attention"]

@@ -1,0 +1,184 @@
+// C ABI of the Adamas decode path: host-side argument checks, then dispatch.
+// Every check runs before any launch; a rejected call launches nothing.
+#include <cmath>
+#include <cstring>
+
+#include "adamas_internal.cuh"
+
+namespace adamas {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int current_device_sms(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev_out) *dev_out = dev;
+  return sms;
+}
+
+}  // namespace adamas
+
+using namespace adamas;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool good_dtype(adamas_dtype dt) { return dt == ADAMAS_F32 || dt == ADAMAS_BF16; }
+bool good_t(float t) { return std::isfinite(t) && t >= 0.0f; }
+bool good_group(int Hq, int Hkv) {
+  if (Hkv <= 0 || Hq <= 0 || Hq % Hkv) return false;
+  const int G = Hq / Hkv;
+  return G == 1 || G == 2 || G == 4 || G == 8;
+}
+adamas_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ADAMAS_OK : ADAMAS_ERR_CUDA; }
+
+// Shared checks of the decode / select entry points.
+adamas_status check_decode_sizes(int B, int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                 int k) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || L <= 0 || k <= 0) return ADAMAS_ERR_INVALID_ARG;
+  if (L > Lmax) return ADAMAS_ERR_INVALID_ARG;
+  if (Hq % Hkv) return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!good_group(Hq, Hkv)) return ADAMAS_ERR_UNSUPPORTED;
+  if (int64_t(B) * Hkv > (1 << 24) || Lmax > (int64_t(1) << 40)) return ADAMAS_ERR_UNSUPPORTED;
+  return ADAMAS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* adamas_status_string(adamas_status s) {
+  switch (s) {
+    case ADAMAS_OK: return "ok";
+    case ADAMAS_ERR_INVALID_ARG: return "invalid argument";
+    case ADAMAS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ADAMAS_ERR_CUDA: return "CUDA error";
+    case ADAMAS_ERR_TIMEOUT: return "a bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+int adamas_abi_version(void) { return 1; }
+
+adamas_status adamas_encode_keys(const void* k_cache, adamas_dtype dt, int B, int Hkv, int d,
+                                 int64_t Lmax, int64_t pos0, int64_t n_new, float t,
+                                 uint8_t* codes, cudaStream_t stream) {
+  if (!k_cache || !codes || !good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || Lmax <= 0 || pos0 < 0 || n_new <= 0 || pos0 + n_new > Lmax)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!aligned(k_cache, 16) || !aligned(codes, 16)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_encode_rows(k_cache, dt, codes, int64_t(B) * Hkv * n_new, n_new, Lmax,
+                                      pos0, t, stream));
+}
+
+adamas_status adamas_encode_queries(const void* q, adamas_dtype dt, int B, int Hq, int d,
+                                    float t, uint8_t* qcodes, cudaStream_t stream) {
+  if (!q || !qcodes || !good_dtype(dt) || !good_t(t) || B <= 0 || Hq <= 0)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(qcodes, 16)) return ADAMAS_ERR_INVALID_ARG;
+  const int64_t n = int64_t(B) * Hq;
+  return from_cuda(launch_encode_rows(q, dt, qcodes, n, n, 0, 0, t, stream));
+}
+
+size_t adamas_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k) {
+  if (check_decode_sizes(B, Hq, Hkv, d, L, L, k) != ADAMAS_OK) return 0;
+  return decode_workspace_bytes(B, Hq, Hkv, L, k);
+}
+
+adamas_status adamas_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!ws || ws_bytes == 0) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, stream));
+}
+
+adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!ws || ws_bytes < 256) return ADAMAS_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  const uint8_t* p = static_cast<const uint8_t*>(ws) + decode_workspace_error_offset();
+  if (cudaMemcpyAsync(&word, p, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return ADAMAS_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
+  return word ? ADAMAS_ERR_TIMEOUT : ADAMAS_OK;
+}
+
+adamas_status adamas_decode_plan(int B, int Hq, int Hkv, int d, int64_t L, int k, int* ctas,
+                                 int* cluster, int64_t* tokens_per_cta, int* smem_bytes) {
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, L, L, k);
+  if (s != ADAMAS_OK) return s;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (ctas) *ctas = p.grid;
+  if (cluster) *cluster = p.cluster;
+  if (tokens_per_cta) *tokens_per_cta = p.keys_per_cta;
+  if (smem_bytes) *smem_bytes = int(p.smem);
+  return ADAMAS_OK;
+}
+
+adamas_status adamas_decode_step(const void* q, const void* k_cache, const void* v_cache,
+                                 const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                 int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
+                                 void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                 float* out, cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !codes || !workspace || !out) return ADAMAS_ERR_INVALID_ARG;
+  if (!good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(codes, 16) ||
+      !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv, Lmax, L,
+                                 k, t, workspace, idx_out, out, p, stream));
+}
+
+adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, int B, int Hq,
+                                 int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
+                                 size_t ws_bytes, int32_t* idx_out, cudaStream_t stream) {
+  if (!qcodes || !codes || !workspace || !idx_out) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, kD, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(qcodes, 16) || !aligned(codes, 16) || !aligned(workspace, 256) ||
+      !aligned(idx_out, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_decode(nullptr, qcodes, nullptr, nullptr, codes, ADAMAS_BF16, B, Hq,
+                                 Hkv, Lmax, L, k, 0.0f, workspace, idx_out, nullptr, p, stream));
+}
+
+size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff) {
+  if (B <= 0 || Hq <= 0 || k_eff <= 0) return 0;
+  return attention_workspace_bytes(B, Hq, k_eff);
+}
+
+adamas_status adamas_sparse_attention(const void* q, const void* k_cache, const void* v_cache,
+                                      adamas_dtype dt, const int32_t* idx, int B, int Hq,
+                                      int Hkv, int d, int64_t Lmax, int k_eff, void* workspace,
+                                      size_t ws_bytes, float* out, cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !idx || !workspace || !out || !good_dtype(dt))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || k_eff <= 0 || Hq % Hkv)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(idx, 4) || !aligned(workspace, 256))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (ws_bytes < attention_workspace_bytes(B, Hq, k_eff)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_sparse_attention(q, k_cache, v_cache, dt, idx, B, Hq, Hkv, Lmax, k_eff,
+                                           workspace, out, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,385 @@
+// Internal device helpers of the Adamas decode path (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "adamas.h"
+
+namespace adamas {
+
+constexpr int kD = 128;                 // head dimension
+constexpr int kCodeBytes = kD / 4;      // 32 B of 2-bit codes per vector
+constexpr int kNBins = 3 * kD + 1;      // Manhattan distances 0..384
+constexpr int kBinStride = 388;         // padded histogram row
+constexpr int kPartStride = 132;        // m, l, 2 pad, acc[128] (floats)
+
+// error word bits (workspace header)
+constexpr uint32_t kErrBarrier = 1u;
+constexpr uint32_t kErrCopy = 2u;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
+
+// ----------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (16-B aligned,
+// bytes a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase; records kErrCopy and returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(err, kErrCopy);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Grid-wide barrier for a cooperative launch (all CTAs co-resident).  Sense by
+// generation counter; the arrival counter returns to zero, so the workspace stays
+// reusable.  Bounded: gives up after kWaitLimitNs and records kErrBarrier.
+__device__ __forceinline__ void grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks,
+                                             uint32_t* err) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t g0 = ld_acquire_gpu(gen);
+    __threadfence();
+    const uint32_t arrived = atomicAdd(count, 1u) + 1u;
+    if (arrived == nblocks) {
+      atomicExch(count, 0u);
+      __threadfence();
+      st_release_gpu(gen, g0 + 1u);
+    } else {
+      const unsigned long long t0 = globaltimer_ns();
+      while (ld_acquire_gpu(gen) == g0) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(err, kErrBarrier);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+// ----------------------------------------------------------- element loading
+// Lane l of a warp owns elements 4l .. 4l+3 of a 128-vector.
+__device__ __forceinline__ void load4(const float* row, int lane, float v[4]) {
+  const float4 x = __ldg(reinterpret_cast<const float4*>(row) + lane);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+
+__device__ __forceinline__ void load4(const __nv_bfloat16* row, int lane, float v[4]) {
+  const uint2 x = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+  bf16x2_to_f32(x.x, v[0], v[1]);
+  bf16x2_to_f32(x.y, v[2], v[3]);
+}
+
+// Raw 4-element chunks kept undecoded while loads are in flight.
+template <typename T> struct Raw4;
+template <> struct Raw4<float> {
+  using type = float4;
+  static __device__ __forceinline__ type load(const float* row, int lane) {
+    return __ldg(reinterpret_cast<const float4*>(row) + lane);
+  }
+  static __device__ __forceinline__ void decode(const type& x, float v[4]) {
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  }
+};
+template <> struct Raw4<__nv_bfloat16> {
+  using type = uint2;
+  static __device__ __forceinline__ type load(const __nv_bfloat16* row, int lane) {
+    return __ldg(reinterpret_cast<const uint2*>(row) + lane);
+  }
+  static __device__ __forceinline__ void decode(const type& x, float v[4]) {
+    bf16x2_to_f32(x.x, v[0], v[1]);
+    bf16x2_to_f32(x.y, v[2], v[3]);
+  }
+};
+
+// ------------------------------------------------------------ FWHT + codes
+// Orthonormal fast Walsh–Hadamard transform of one 128-vector held by a warp
+// (lane l: elements 4l..4l+3), natural (Sylvester) order, fp32.  Index bits 0-1
+// are butterflied inside the lane, bits 2-6 across lanes with xor-shuffles.
+// Returns the lane's byte of the packed code: 4 coordinates, 2 bits each,
+// coordinate 4l+r at bits 2r, code = [y >= -t] + [y >= 0] + [y >= t].
+__device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane) {
+  const float a0 = v[0] + v[1], a1 = v[0] - v[1];
+  const float a2 = v[2] + v[3], a3 = v[2] - v[3];
+  v[0] = a0 + a2; v[1] = a1 + a3; v[2] = a0 - a2; v[3] = a1 - a3;
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[r], s);
+      v[r] = upper ? (o - v[r]) : (v[r] + o);
+    }
+  }
+  const float inv_sqrt_d = 0.088388347648318440550f;   // 1 / sqrt(128)
+  uint32_t byte = 0;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float y = v[r] * inv_sqrt_d;
+    v[r] = y;
+    const uint32_t c = (uint32_t)(y >= -t) + (uint32_t)(y >= 0.0f) + (uint32_t)(y >= t);
+    byte |= c << (2 * r);
+  }
+  return byte;
+}
+
+// --------------------------------------------------------- code arithmetic
+// Thermometer form of a word of 16 packed codes: for code c = 2h + l the field
+// becomes (odd, even) = ([c >= 3], [c >= 1]).
+__device__ __forceinline__ uint32_t therm13(uint32_t w) {
+  const uint32_t d = (w >> 1) & ~w & 0x55555555u;      // h & ~l, at the even bit
+  return w ^ d ^ (d << 1);
+}
+// [c >= 2] of two words, the first at even bits, the second at odd bits.
+__device__ __forceinline__ uint32_t therm2(uint32_t w0, uint32_t w1) {
+  return ((w0 >> 1) & 0x55555555u) | (w1 & 0xaaaaaaaau);
+}
+
+// Thermometer words of one packed 32-byte code: 8 x therm13 + 4 x therm2.
+struct Therm {
+  uint32_t a[8];
+  uint32_t b[4];
+};
+
+__device__ __forceinline__ void make_therm(const uint32_t w[8], Therm& t) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t.a[i] = therm13(w[i]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t.b[i] = therm2(w[2 * i], w[2 * i + 1]);
+}
+
+// Manhattan distance of two code vectors from their thermometer words:
+// |a - b| = [a>=1]^[b>=1] + [a>=2]^[b>=2] + [a>=3]^[b>=3] per coordinate.
+__device__ __forceinline__ uint32_t therm_dist(const Therm& k, const Therm& q) {
+  uint32_t s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s0 += __popc(k.a[2 * i] ^ q.a[2 * i]);
+    s1 += __popc(k.a[2 * i + 1] ^ q.a[2 * i + 1]);
+    s2 += __popc(k.b[i] ^ q.b[i]);
+  }
+  return s0 + s1 + s2;
+}
+
+// Same distance with one carry-save level: the 12 XOR words are added bitwise three
+// at a time (sum word = a^b^c, carry word = majority(a,b,c), both single LOP3s),
+// so 8 popcounts replace 12.  POPC issues at a quarter of the integer-logic rate on
+// sm_100, so this moves work from the saturated popcount pipe to the logic pipe.
+__device__ __forceinline__ uint32_t therm_dist_csa(const Therm& k, const Therm& q) {
+  uint32_t x[12];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = k.a[i] ^ q.a[i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[8 + i] = k.b[i] ^ q.b[i];
+  uint32_t ones = 0, twos = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t a = x[3 * j], b = x[3 * j + 1], c = x[3 * j + 2];
+    ones += __popc(a ^ b ^ c);
+    twos += __popc((a & b) | (c & (a | b)));
+  }
+  return ones + 2u * twos;
+}
+
+// ---------------------------------------------------------- warp utilities
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Online-softmax state of one (warp, head): scores are kept in the log2 domain.
+struct SoftmaxState {
+  float m;       // running max of scaled scores (log2 domain)
+  float l;       // running sum of exp2(s - m)
+  float acc[4];  // lane's 4 output coordinates, unnormalised
+  __device__ __forceinline__ void init() {
+    m = -INFINITY; l = 0.f;
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  }
+};
+
+// Gathers up to `n` rows (positions from `pos_of(j)` for j = j0, j0+step, ...)
+// and folds them into `st`.  K/V row r of this (batch, kv head) starts at
+// base + r * kD.  Four rows are in flight per warp per batch.
+template <typename T, typename PosFn>
+__device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
+                                            const T* __restrict__ vbase, int n, int j0,
+                                            int step, PosFn pos_of, const float q[4],
+                                            float scale_log2, int lane, SoftmaxState& st) {
+  using R = Raw4<T>;
+  for (int j = j0; j < n; j += 4 * step) {
+    typename R::type kr[4], vr[4];
+    bool valid[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int jj = j + u * step;
+      valid[u] = jj < n;
+      if (valid[u]) {
+        const int64_t pos = pos_of(jj);
+        kr[u] = R::load(kbase + pos * kD, lane);
+        vr[u] = R::load(vbase + pos * kD, lane);
+      }
+    }
+    float s[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float kv[4];
+      if (valid[u]) {
+        R::decode(kr[u], kv);
+        s[u] = q[0] * kv[0] + q[1] * kv[1] + q[2] * kv[2] + q[3] * kv[3];
+      } else {
+        s[u] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+    }
+    float mx = st.m;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      s[u] = valid[u] ? s[u] * scale_log2 : -INFINITY;
+      mx = fmaxf(mx, s[u]);
+    }
+    const float corr = exp2f(st.m - mx);   // st.m = -inf -> 0
+    st.l *= corr;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) st.acc[r] *= corr;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (valid[u]) {
+        const float p = exp2f(s[u] - mx);
+        float vv[4];
+        R::decode(vr[u], vv);
+        st.l += p;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) st.acc[r] = fmaf(p, vv[r], st.acc[r]);
+      }
+    }
+    st.m = mx;
+  }
+}
+
+// Merge two softmax partials (m, l, acc) into (M, Lsum, A) accumulators.
+__device__ __forceinline__ void merge_into(float m, float l, float a, float& M, float& Ls,
+                                           float& A) {
+  if (l == 0.f) return;
+  if (m > M) {
+    const float c = exp2f(M - m);
+    Ls = Ls * c + l;
+    A = A * c + a;
+    M = m;
+  } else {
+    const float c = exp2f(m - M);
+    Ls += l * c;
+    A += a * c;
+  }
+}
+
+// ------------------------------------------------------------- host side
+int current_device_sms(int* dev_out);
+size_t align_up(size_t x, size_t a);
+
+// Launch plan of the fused decode kernel (one thread-block cluster per unit).
+struct Plan {
+  int grid;              // CTAs = units x cluster
+  int cluster;           // CTAs per (batch, kv head) unit
+  int waves;             // modelled waves of clusters over the device
+  int64_t keys_per_cta;  // R = ceil(L / cluster)
+  int list_cap;          // selected-position slots per head per CTA
+  size_t smem;           // dynamic shared memory bytes
+};
+bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, Plan& p);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k);
+size_t decode_workspace_error_offset();
+cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
+                          const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
+                          int64_t Lmax, int64_t L, int kk, float t, void* ws, int32_t* idx_out,
+                          float* out, const Plan& p, cudaStream_t stream);
+cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
+                               int64_t per, int64_t stride, int64_t off, float t,
+                               cudaStream_t stream);
+size_t attention_workspace_bytes(int B, int Hq, int k_eff);
+cudaError_t launch_sparse_attention(const void* q, const void* k, const void* v,
+                                    adamas_dtype dt, const int32_t* idx, int B, int Hq,
+                                    int Hkv, int64_t Lmax, int k_eff, void* ws, float* out,
+                                    cudaStream_t stream);
+
+}  // namespace adamas

@@ -1,0 +1,644 @@
+// Fused Adamas decode step: ONE launch of a thread-block-cluster kernel runs
+//   query encode -> distance scan -> exact per-head top-k -> gather attention
+//   (one split per CTA) -> combine of the splits,
+// with every cross-CTA exchange in distributed shared memory.
+//
+// Method: "Adamas: Hadamard Sparse Attention for Efficient Long-Context
+// Inference" — v2 abstract (compact 2-bit codes, distance-based top-k, gather of
+// the original KV states for sparse attention), v1 abstract (Manhattan distance).
+//
+// Work split.  A (batch, kv head) pair is a "unit".  Each unit gets one cluster
+// of CS CTAs (CS <= 16, one CTA per SM); CTA r of the cluster owns key positions
+// [r*R, min(L, (r+1)*R)), R = ceil(L / CS).  Clusters are independent, so more
+// units than fit at once simply run in waves.
+//
+// Exact top-k with ties to the lower position.  Distances are integers 0..384.
+// Each CTA keeps its distances in shared memory and builds, per query head, a
+// 385-bin histogram that it turns into a cumulative one.  After a cluster barrier
+// every CTA reads its peers' cumulative histograms through distributed shared
+// memory — first at 30 coarse bins, then at 14 bins around the crossing — which
+// gives the k-th distance D*, how many tokens of lower-ranked CTAs are selected,
+// and how many of its own D*-ties it takes.  One block scan in position order then
+// emits its selected positions.  The key codes cross HBM exactly once, and no
+// global-memory atomic, barrier or scratch is involved.
+//
+// Attention.  Each CTA gathers the original K/V rows it selected (one split of
+// the unit's softmax) and stores its partial (m, l, acc[128]) per head into the
+// shared memory of cluster rank 0; after a second cluster barrier rank 0 merges
+// the CS partials and writes the output.
+#include <algorithm>
+#include <mutex>
+
+#include <cooperative_groups.h>
+
+#include "adamas_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace adamas {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = 512;      // keys per bulk copy (16 KiB of codes)
+constexpr int kStages = 4;       // bulk-copy ring depth
+constexpr int kMaxCluster = 16;  // non-portable cluster size limit
+constexpr int kCoarse = 13;      // bins per coarse chunk of the D* search (30 chunks)
+constexpr int kRound = kThreads * 32;   // tokens per select round (32 per thread)
+
+__host__ __device__ inline int dist_stride(int R) { return (R + 7) & ~7; }
+
+struct DecodeArgs {
+  const void* q;             // [B][Hq][128] (encode mode) or nullptr
+  const uint8_t* qcodes;     // [B][Hq][32] (select mode) or nullptr
+  const void* k;             // [B][Hkv][Lmax][128]
+  const void* v;
+  const uint8_t* codes;      // [B][Hkv][Lmax][32]
+  int B, Hq, Hkv;
+  int64_t Lmax, L;
+  int k_eff;
+  float t;
+  float scale_log2;
+  int32_t* idx_out;          // [B][Hq][k_eff] or nullptr
+  float* out;                // [B][Hq][128] or nullptr (select mode)
+  uint32_t* err;             // device error word
+  int cluster;               // CTAs per unit
+  int keys_per_cta;          // R
+  int list_cap;
+  int attend;
+};
+
+struct SmemLayout {
+  size_t ring, mbar, hist, dist, list, qf, qc, qth, scan, merge, info, misc, total;
+};
+
+__host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline SmemLayout make_layout(int G, int R, int list_cap, int CS) {
+  SmemLayout s;
+  size_t o = 0;
+  const size_t ring = size_t(kStages) * kChunk * kCodeBytes;
+  const size_t part = size_t(CS) * G * kPartStride * 4;   // rank 0 receives the partials
+  s.ring = o;  o = al(o + (ring > part ? ring : part), 128);
+  s.mbar = o;  o = al(o + 8 * kStages, 128);
+  s.hist = o;  o = al(o + size_t(G) * kBinStride * 4, 128);
+  s.dist = o;  o = al(o + size_t(G) * dist_stride(R) * 2, 128);
+  s.list = o;  o = al(o + size_t(G) * list_cap * 2, 128);
+  s.qf = o;    o = al(o + size_t(G) * kD * 4, 128);
+  s.qc = o;    o = al(o + size_t(G) * kCodeBytes, 128);
+  s.qth = o;   o = al(o + size_t(G) * 12 * 4, 128);
+  s.scan = o;  o = al(o + size_t(kWarps + 1) * G * 4, 128);
+  s.merge = o; o = al(o + size_t(kWarps) * kPartStride * 4, 128);
+  s.info = o;  o = al(o + size_t(G) * 8 * 4, 128);
+  s.misc = o;  o = al(o + 128, 128);
+  s.total = o;
+  return s;
+}
+
+// Exclusive prefix over the block (thread order) of G counters per thread; also
+// returns the block totals.  scan holds (kWarps + 1) x G words.
+template <int G>
+__device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t (&total)[G],
+                                                     uint32_t* scan, int lane, int warp) {
+  uint32_t inc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    uint32_t x = v[g];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    inc[g] = x;
+    if (lane == 31) scan[warp * G + g] = x;
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const uint32_t own = lane < kWarps ? scan[lane * G + g] : 0u;
+      uint32_t x = own;
+#pragma unroll
+      for (int o = 1; o < kWarps; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane < kWarps) scan[lane * G + g] = x - own;
+      if (lane == kWarps - 1) scan[kWarps * G + g] = x;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    v[g] = scan[warp * G + g] + inc[g] - v[g];
+    total[g] = scan[kWarps * G + g];
+  }
+  __syncthreads();
+}
+
+template <int G, typename T>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = a.cluster;
+  const int rank = int(cluster.block_rank());
+  const SmemLayout lo = make_layout(G, a.keys_per_cta, a.list_cap, CS);
+  uint8_t* ring = smem + lo.ring;
+  float* part = reinterpret_cast<float*>(smem + lo.ring);           // [CS][G][kPartStride]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + lo.hist);    // [G][kBinStride]
+  uint16_t* dist = reinterpret_cast<uint16_t*>(smem + lo.dist);    // [G][RS]
+  uint16_t* list = reinterpret_cast<uint16_t*>(smem + lo.list);    // [G][list_cap]
+  float* qf = reinterpret_cast<float*>(smem + lo.qf);              // [G][128]
+  uint8_t* qc = smem + lo.qc;                                       // [G][32]
+  uint32_t* qth = reinterpret_cast<uint32_t*>(smem + lo.qth);      // [G][12]
+  uint32_t* scan = reinterpret_cast<uint32_t*>(smem + lo.scan);    // [kWarps][G]
+  float* merge = reinterpret_cast<float*>(smem + lo.merge);        // [kWarps][kPartStride]
+  int* info = reinterpret_cast<int*>(smem + lo.info);              // [G][8]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int unit = blockIdx.x / CS;
+  const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int64_t L = a.L;
+  const int R = a.keys_per_cta;
+  const int RS = dist_stride(R);
+  const int64_t p0 = int64_t(rank) * R;
+  const int n = int(max(int64_t(0), min(int64_t(R), L - p0)));   // keys of this CTA
+  const int nch = (n + kChunk - 1) / kChunk;
+  const uint8_t* codes = a.codes + (int64_t(unit) * a.Lmax + p0) * kCodeBytes;
+
+  // ---- issue the code copies first: HBM traffic starts before anything else
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
+    fence_mbar_init();
+    for (int qi = 0; qi < min(nch, kStages); ++qi) {
+      const int keys = min(kChunk, n - qi * kChunk);
+      mbar_expect_tx(&mbar[qi], uint32_t(keys * kCodeBytes));
+      bulk_g2s(ring + size_t(qi) * kChunk * kCodeBytes,
+               codes + int64_t(qi) * kChunk * kCodeBytes, uint32_t(keys * kCodeBytes), &mbar[qi]);
+    }
+  }
+
+  // ---- prologue: zero histograms, encode (or fetch) the G query codes
+  for (int i = tid; i < G * kBinStride; i += kThreads) hist[i] = 0u;
+  if (warp < G) {
+    const int g = warp, h = kvh * G + g;
+    if (a.qcodes != nullptr) {
+      qc[g * kCodeBytes + lane] = a.qcodes[(int64_t(b) * a.Hq + h) * kCodeBytes + lane];
+    } else {
+      float v[4];
+      load4(static_cast<const T*>(a.q) + (int64_t(b) * a.Hq + h) * kD, lane, v);
+      float* qrow = qf + g * kD + 4 * lane;
+      qrow[0] = v[0]; qrow[1] = v[1]; qrow[2] = v[2]; qrow[3] = v[3];
+      qc[g * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(v, a.t, lane));
+    }
+  }
+  __syncthreads();
+  if (tid < G) {
+    const uint32_t* wq = reinterpret_cast<const uint32_t*>(qc + tid * kCodeBytes);
+    uint32_t wd[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wd[i] = wq[i];
+    Therm th;
+    make_therm(wd, th);
+    uint32_t* dst = qth + tid * 12;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = th.a[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[8 + i] = th.b[i];
+  }
+  __syncthreads();
+
+  // ---- distance scan: one key per thread per chunk, G heads per key
+  {
+    constexpr int GR = G > 4 ? 4 : G;
+    Therm qreg[GR];
+    if constexpr (G <= 4) {
+#pragma unroll
+      for (int g = 0; g < GR; ++g) {
+        const uint32_t* s = qth + g * 12;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qreg[g].a[i] = s[i];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qreg[g].b[i] = s[8 + i];
+      }
+    }
+    const int swz = (tid >> 2) & 1;   // conflict-free 2 x 16 B reads of a 32 B code
+    for (int qi = 0; qi < nch; ++qi) {
+      const int slot = qi % kStages;
+      mbar_wait_bounded(&mbar[slot], uint32_t(qi / kStages) & 1u, a.err);
+      const int r = qi * kChunk + tid;
+      if (r < n) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            ring + (size_t(slot) * kChunk + tid) * kCodeBytes);
+        const uint4 xa = src[swz], xb = src[swz ^ 1];
+        const uint4 x0 = swz ? xb : xa, x1 = swz ? xa : xb;
+        const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        Therm kt;
+        make_therm(wd, kt);
+#pragma unroll
+        for (int g0 = 0; g0 < G; g0 += GR) {
+          if constexpr (G > 4) {
+#pragma unroll
+            for (int g = 0; g < GR; ++g) {
+              const uint4* s = reinterpret_cast<const uint4*>(qth + (g0 + g) * 12);
+              const uint4 p0v = s[0], p1v = s[1], p2v = s[2];
+              qreg[g].a[0] = p0v.x; qreg[g].a[1] = p0v.y; qreg[g].a[2] = p0v.z; qreg[g].a[3] = p0v.w;
+              qreg[g].a[4] = p1v.x; qreg[g].a[5] = p1v.y; qreg[g].a[6] = p1v.z; qreg[g].a[7] = p1v.w;
+              qreg[g].b[0] = p2v.x; qreg[g].b[1] = p2v.y; qreg[g].b[2] = p2v.z; qreg[g].b[3] = p2v.w;
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < GR; ++g) {
+            const uint32_t dd = therm_dist_csa(kt, qreg[g]);
+            dist[size_t(g0 + g) * RS + r] = static_cast<uint16_t>(dd);
+            atomicAdd(&hist[(g0 + g) * kBinStride + dd], 1u);
+          }
+        }
+      }
+      __syncthreads();
+      if (tid == 0 && qi + kStages < nch) {
+        const int nx = qi + kStages;
+        const int keys = min(kChunk, n - nx * kChunk);
+        mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes));
+        bulk_g2s(ring + size_t(slot) * kChunk * kCodeBytes,
+                 codes + int64_t(nx) * kChunk * kCodeBytes, uint32_t(keys * kCodeBytes),
+                 &mbar[slot]);
+      }
+    }
+  }
+
+  // ---- histograms -> inclusive cumulative histograms, in place (warp per head)
+  if (warp < G) {
+    uint32_t* row = hist + warp * kBinStride;
+    uint32_t loc[kCoarse];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int i = 0; i < kCoarse; ++i) {
+      const int bin = kCoarse * lane + i;
+      loc[i] = bin < kNBins ? row[bin] : 0u;
+      sum += loc[i];
+    }
+    uint32_t inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    uint32_t run = inc - sum;
+#pragma unroll
+    for (int i = 0; i < kCoarse; ++i) {
+      const int bin = kCoarse * lane + i;
+      run += loc[i];
+      if (bin < kNBins) row[bin] = run;
+    }
+  }
+
+  cluster.sync();   // every CTA's cumulative histograms are complete and visible
+
+  // ---- resolve D*, the count selected in lower-ranked CTAs, and the ties taken
+  if (warp < G) {
+    const int g = warp;
+    const uint32_t ke = uint32_t(a.k_eff);
+    // level 1: cumulative counts of the whole unit at the end of each coarse chunk;
+    // all peer loads are issued before any is summed
+    uint32_t S1 = 0;
+    if (lane < 30) {
+      const int bj = min(kCoarse * lane + kCoarse - 1, kNBins - 1);
+      uint32_t v[kMaxCluster];
+#pragma unroll
+      for (int cc = 0; cc < kMaxCluster; ++cc)
+        v[cc] = cc < CS ? cluster.map_shared_rank(hist, cc)[g * kBinStride + bj] : 0u;
+#pragma unroll
+      for (int cc = 0; cc < kMaxCluster; ++cc) S1 += v[cc];
+    }
+    const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < 30 && S1 >= ke);
+    const int jstar = __ffs(hit1) - 1;   // exists: the last chunk ends at bin 384, count L
+    // level 2: bins 13 j* - 1 .. 13 j* + 12 (lane l -> bin 13 j* - 1 + l)
+    const int d = kCoarse * jstar - 1 + lane;
+    uint32_t S2 = 0, Sb = 0;
+    if (lane < kCoarse + 1 && d >= 0) {
+      const int dd = min(d, kNBins - 1);
+      uint32_t v[kMaxCluster];
+#pragma unroll
+      for (int cc = 0; cc < kMaxCluster; ++cc)
+        v[cc] = cc < CS ? cluster.map_shared_rank(hist, cc)[g * kBinStride + dd] : 0u;
+#pragma unroll
+      for (int cc = 0; cc < kMaxCluster; ++cc) {
+        S2 += v[cc];
+        if (cc < rank) Sb += v[cc];
+      }
+    }
+    const uint32_t hit2 = __ballot_sync(0xffffffffu, lane >= 1 && lane < kCoarse + 1 && S2 >= ke);
+    const int ls = __ffs(hit2) - 1;
+    const int dstar = kCoarse * jstar - 1 + ls;
+    const uint32_t less = __shfl_sync(0xffffffffu, S2, ls - 1);       // unit count d < D*
+    const uint32_t lt_before = __shfl_sync(0xffffffffu, Sb, ls - 1);
+    const uint32_t eq_before = __shfl_sync(0xffffffffu, Sb, ls) - lt_before;
+    const uint32_t* own = hist + g * kBinStride;
+    const uint32_t lt_own = dstar > 0 ? own[dstar - 1] : 0u;
+    const uint32_t eq_own = own[dstar] - lt_own;
+    const uint32_t need = ke - less;                 // ties at D* the unit takes
+    const uint32_t base = lt_before + min(eq_before, need);
+    const uint32_t take = need > eq_before ? min(need - eq_before, eq_own) : 0u;
+    if (lane == 0) {
+      int* in = info + g * 8;
+      in[0] = dstar;
+      in[1] = int(base);
+      in[2] = int(take);
+      in[3] = int(lt_own + take);   // selected in this CTA
+    }
+  }
+  __syncthreads();
+
+  // ---- select, in position order: per round each thread owns up to 32 consecutive
+  // tokens; one pass over the distances builds "< D*" and "== D*" bit masks, one
+  // block scan ranks them, and only the selected bits are then visited
+  {
+    int dstar[G], take[G], base[G], nsel[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int* in = info + g * 8;
+      dstar[g] = in[0];
+      base[g] = in[1];
+      take[g] = in[2];
+      nsel[g] = in[3];
+    }
+    uint32_t carry_lt[G], carry_eq[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) carry_lt[g] = carry_eq[g] = 0;
+    for (int rb = 0; rb < n; rb += kRound) {
+      const int nr = min(kRound, n - rb);
+      const int per = (((nr + kThreads - 1) / kThreads) + 7) & ~7;   // multiple of 8, <= 32
+      const int s0 = rb + tid * per;
+      const int cntv = max(0, min(per, rb + nr - s0));
+      uint32_t ltm[G], eqm[G], cnt[G], tot[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        ltm[g] = eqm[g] = 0;
+        const uint16_t* row = dist + size_t(g) * RS + s0;
+        for (int i8 = 0; i8 < cntv; i8 += 8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(row + i8);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int dv = int((w[j >> 1] >> (16 * (j & 1))) & 0xffffu);
+            const uint32_t bit = (i8 + j < cntv) ? (1u << (i8 + j)) : 0u;
+            if (dv < dstar[g]) ltm[g] |= bit;
+            if (dv == dstar[g]) eqm[g] |= bit;
+          }
+        }
+        cnt[g] = (uint32_t(__popc(ltm[g])) << 16) | uint32_t(__popc(eqm[g]));
+      }
+      block_exclusive_scan<G>(cnt, tot, scan, lane, warp);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int lt_b = int(carry_lt[g] + (cnt[g] >> 16));
+        const int eq_b = int(carry_eq[g] + (cnt[g] & 0xffffu));
+        // this thread's ties that still fit: the lowest (take - eq_b) bits of eqm
+        uint32_t sel_eq = 0;
+        const int te = take[g] - eq_b;
+        if (te > 0) {
+          uint32_t rest = eqm[g];
+          for (int c = 0; c < te && rest; ++c) rest &= rest - 1u;
+          sel_eq = eqm[g] ^ rest;
+        }
+        uint32_t sel = ltm[g] | sel_eq;
+        int rk = lt_b + min(eq_b, take[g]);
+        int32_t* orow = a.idx_out != nullptr
+                            ? a.idx_out + (int64_t(b) * a.Hq + kvh * G + g) * a.k_eff + base[g]
+                            : nullptr;
+        uint16_t* lrow = list + size_t(g) * a.list_cap;
+        while (sel) {
+          const int i = __ffs(sel) - 1;
+          sel &= sel - 1u;
+          const int r = s0 + i;
+          // rk < nsel and base + rk < k_eff hold by construction; the guard keeps a
+          // broken invariant from writing outside the list or the output row
+          if (rk < nsel[g] && base[g] + rk < a.k_eff) {
+            lrow[rk] = static_cast<uint16_t>(r);
+            if (orow) orow[rk] = int32_t(p0 + r);
+          }
+          ++rk;
+        }
+        carry_lt[g] += tot[g] >> 16;
+        carry_eq[g] += tot[g] & 0xffffu;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- attention over the selected rows: this CTA's split of the unit's softmax
+  if (a.attend) {
+    constexpr int WPH = kWarps / G;   // warps per head
+    const int g = warp % G, sub = warp / G;
+    const int nsel = info[g * 8 + 3];
+    const uint16_t* lrow = list + size_t(g) * a.list_cap;
+    const float* qrow = qf + g * kD + 4 * lane;
+    const float qv[4] = {qrow[0], qrow[1], qrow[2], qrow[3]};
+    const T* kb = static_cast<const T*>(a.k) + int64_t(unit) * a.Lmax * kD;
+    const T* vb = static_cast<const T*>(a.v) + int64_t(unit) * a.Lmax * kD;
+    SoftmaxState st;
+    st.init();
+    attend_rows<T>(kb, vb, nsel, sub, WPH, [&](int j) { return p0 + int64_t(lrow[j]); }, qv,
+                   a.scale_log2, lane, st);
+    float* mw = merge + warp * kPartStride;
+    if (lane == 0) { mw[0] = st.m; mw[1] = st.l; }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) mw[4 + 4 * lane + r] = st.acc[r];
+    __syncthreads();
+    float* dstp = cluster.map_shared_rank(part, 0) + size_t(rank) * G * kPartStride;
+    for (int i = tid; i < G * kD; i += kThreads) {
+      const int gg = i / kD, dim = i % kD;
+      float M = -INFINITY, Ls = 0.f, A = 0.f;
+      for (int sw = 0; sw < WPH; ++sw) {
+        const float* mm = merge + (sw * G + gg) * kPartStride;
+        merge_into(mm[0], mm[1], mm[4 + dim], M, Ls, A);
+      }
+      float* prow = dstp + gg * kPartStride;
+      if (dim == 0) { prow[0] = M; prow[1] = Ls; }
+      prow[4 + dim] = A;
+    }
+  }
+
+  cluster.sync();   // partials are in rank 0; no CTA reads a peer's memory after this
+
+  if (a.attend && rank == 0) {
+    for (int i = tid; i < G * kD; i += kThreads) {
+      const int gg = i / kD, dim = i % kD;
+      float M = -INFINITY;
+      for (int cc = 0; cc < CS; ++cc) M = fmaxf(M, part[(cc * G + gg) * kPartStride]);
+      float Ls = 0.f, A = 0.f;
+      for (int cc = 0; cc < CS; ++cc) {
+        const float* prow = part + (cc * G + gg) * kPartStride;
+        const float e = exp2f(prow[0] - M);     // empty split: m = -inf -> 0
+        Ls = fmaf(prow[1], e, Ls);
+        A = fmaf(prow[4 + dim], e, A);
+      }
+      a.out[(int64_t(b) * a.Hq + kvh * G + gg) * kD + dim] = A / Ls;
+    }
+  }
+}
+
+// ------------------------------------------------------------------- host side
+static int max_smem_optin(int dev) {
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 232448;
+  }
+  return v;
+}
+
+template <int G, typename T>
+static cudaError_t prepare_kernel() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    err = cudaFuncSetAttribute(decode_kernel<G, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               max_smem_optin(dev));
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(decode_kernel<G, T>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  });
+  return err;
+}
+
+template <int G, typename T>
+static int active_clusters_g(int cs, size_t smem) {
+  if (prepare_kernel<G, T>() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, T>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return nclusters;
+}
+
+static int active_clusters(int G, int cs, size_t smem) {
+  switch (G) {
+    case 1: return active_clusters_g<1, __nv_bfloat16>(cs, smem);
+    case 2: return active_clusters_g<2, __nv_bfloat16>(cs, smem);
+    case 4: return active_clusters_g<4, __nv_bfloat16>(cs, smem);
+    case 8: return active_clusters_g<8, __nv_bfloat16>(cs, smem);
+  }
+  return 0;
+}
+
+// Chooses the cluster size: among sizes whose shared memory fits (and, on a device,
+// whose clusters can be scheduled), the one with the least modelled time
+// waves x (per-key scan cost x keys per CTA + fixed per-wave latency).
+bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int smem_cap,
+                      bool query_device, Plan& p) {
+  const int G = Hq / Hkv;
+  const int64_t U = int64_t(B) * Hkv;
+  const int64_t k_eff = std::min<int64_t>(k, L);
+  double best = 0;
+  bool found = false;
+  for (int cs = 1; cs <= kMaxCluster; ++cs) {
+    const int64_t R = (L + cs - 1) / cs;
+    if (R > 65535) continue;                       // positions in a CTA are 16-bit
+    if (cs > 1 && (L + R - 1) / R < cs) continue;  // an all-empty tail CTA: use fewer
+    const int list_cap = int(std::max<int64_t>(1, std::min<int64_t>(R, k_eff)));
+    const size_t smem = make_layout(G, int(R), list_cap, cs).total;
+    if (smem > size_t(smem_cap)) continue;
+    int conc_clusters = sms / cs;
+    if (query_device) conc_clusters = active_clusters(G, cs, smem);
+    if (conc_clusters < 1) continue;
+    const int64_t total = U * cs;
+    const int64_t conc = int64_t(conc_clusters) * cs;
+    const int64_t waves = (total + conc - 1) / conc;
+    const double per_key_ns = 0.45 * G + 0.35;
+    const double cost = double(waves) * (per_key_ns * double(R) + 6000.0);
+    if (!found || cost < best) {
+      best = cost;
+      found = true;
+      p.grid = int(total);
+      p.cluster = cs;
+      p.keys_per_cta = R;
+      p.list_cap = list_cap;
+      p.smem = smem;
+      p.waves = int(waves);
+    }
+  }
+  return found && p.grid > 0 && int64_t(p.grid) == U * p.cluster && U * p.cluster < (1ll << 31);
+}
+
+bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, Plan& p) {
+  int dev = 0;
+  const int sms = current_device_sms(&dev);
+  if (sms <= 0) {
+    // no device visible: plan for a 148-SM part with the sm_100 shared-memory cap
+    return make_decode_plan(B, Hq, Hkv, L, k, 148, 232448, false, p);
+  }
+  return make_decode_plan(B, Hq, Hkv, L, k, sms, max_smem_optin(dev), true, p);
+}
+
+// The decode workspace only carries the device error word (bounded copy waits).
+size_t decode_workspace_bytes(int, int, int, int64_t, int) { return 256; }
+size_t decode_workspace_error_offset() { return 8; }
+
+template <int G, typename T>
+static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t stream) {
+  const cudaError_t e = prepare_kernel<G, T>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<G, T>, a);
+}
+
+template <typename T>
+static cudaError_t launch_t(int G, const DecodeArgs& a, const Plan& p, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_g<1, T>(a, p, s);
+    case 2: return launch_g<2, T>(a, p, s);
+    case 4: return launch_g<4, T>(a, p, s);
+    case 8: return launch_g<8, T>(a, p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
+                          const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
+                          int64_t Lmax, int64_t L, int kk, float t, void* ws,
+                          int32_t* idx_out, float* out, const Plan& p, cudaStream_t stream) {
+  const int G = Hq / Hkv;
+  DecodeArgs a;
+  a.q = q; a.qcodes = qcodes; a.k = k; a.v = v; a.codes = codes;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lmax = Lmax; a.L = L;
+  a.k_eff = int(std::min<int64_t>(kk, L));
+  a.t = t;
+  a.scale_log2 = float(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
+  a.idx_out = idx_out; a.out = out;
+  a.err = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + decode_workspace_error_offset());
+  a.cluster = p.cluster;
+  a.keys_per_cta = int(p.keys_per_cta);
+  a.list_cap = p.list_cap;
+  a.attend = out != nullptr ? 1 : 0;
+  if (dt == ADAMAS_F32) return launch_t<float>(G, a, p, stream);
+  return launch_t<__nv_bfloat16>(G, a, p, stream);
+}
+
+}  // namespace adamas

@@ -127,6 +127,15 @@ __device__ __forceinline__ void grid_barrier(uint32_t* count, uint32_t* gen, uin
   __syncthreads();
 }
 
+// L2 prefetch of one 128-element row (256 B bf16 / 512 B fp32), 128 B per line.
+template <typename T>
+__device__ __forceinline__ void prefetch_row_l2(const T* row) {
+  const char* p = reinterpret_cast<const char*>(row);
+#pragma unroll
+  for (int o = 0; o < int(kD * sizeof(T)); o += 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p + o));
+}
+
 // ----------------------------------------------------------- element loading
 // Lane l of a warp owns elements 4l .. 4l+3 of a 128-vector.
 __device__ __forceinline__ void load4(const float* row, int lane, float v[4]) {
@@ -364,6 +373,7 @@ struct Plan {
   int waves;             // modelled waves of clusters over the device
   int64_t keys_per_cta;  // R = ceil(L / cluster)
   int list_cap;          // selected-position slots per head per CTA
+  int stages;            // bulk-copy ring depth
   size_t smem;           // dynamic shared memory bytes
 };
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, Plan& p);

@@ -39,10 +39,13 @@ namespace adamas {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kChunk = 512;      // keys per bulk copy (16 KiB of codes)
-constexpr int kStages = 4;       // bulk-copy ring depth
+constexpr int kChunk = kThreads;  // keys per bulk copy (16 KiB of codes), one per thread
+constexpr int kMaxStages = 4;    // bulk-copy ring depth (runtime: 2..4, as shared memory allows)
 constexpr int kMaxCluster = 16;  // non-portable cluster size limit
 constexpr int kCoarse = 13;      // bins per coarse chunk of the D* search (30 chunks)
+constexpr int kNCoarse = 30;     // coarse chunks (30 x 13 >= 385 bins)
+constexpr int kCoarseRow = 32;   // coarse counts per (CTA, head), padded to 128 B
+constexpr int kFine = 20;        // bins of the fine window (5 x 16 B)
 constexpr int kRound = kThreads * 32;   // tokens per select round (32 per thread)
 
 __host__ __device__ inline int dist_stride(int R) { return (R + 7) & ~7; }
@@ -64,23 +67,27 @@ struct DecodeArgs {
   int cluster;               // CTAs per unit
   int keys_per_cta;          // R
   int list_cap;
+  int stages;                // bulk-copy ring depth
   int attend;
 };
 
 struct SmemLayout {
-  size_t ring, mbar, hist, dist, list, qf, qc, qth, scan, merge, info, misc, total;
+  size_t ring, mbar, hist, coarse, fine, dist, list, qf, qc, qth, scan, merge, info, misc, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SmemLayout make_layout(int G, int R, int list_cap, int CS) {
+__host__ __device__ inline SmemLayout make_layout(int G, int R, int list_cap, int CS,
+                                                 int stages) {
   SmemLayout s;
   size_t o = 0;
-  const size_t ring = size_t(kStages) * kChunk * kCodeBytes;
+  const size_t ring = size_t(stages) * kChunk * kCodeBytes;
   const size_t part = size_t(CS) * G * kPartStride * 4;   // rank 0 receives the partials
   s.ring = o;  o = al(o + (ring > part ? ring : part), 128);
-  s.mbar = o;  o = al(o + 8 * kStages, 128);
+  s.mbar = o;  o = al(o + 8 * kMaxStages, 128);
   s.hist = o;  o = al(o + size_t(G) * kBinStride * 4, 128);
+  s.coarse = o; o = al(o + size_t(CS) * G * kCoarseRow * 4, 128);   // pushed by the peers
+  s.fine = o;  o = al(o + size_t(CS) * G * kFine * 4, 128);         // pulled from the peers
   s.dist = o;  o = al(o + size_t(G) * dist_stride(R) * 2, 128);
   s.list = o;  o = al(o + size_t(G) * list_cap * 2, 128);
   s.qf = o;    o = al(o + size_t(G) * kD * 4, 128);
@@ -88,10 +95,18 @@ __host__ __device__ inline SmemLayout make_layout(int G, int R, int list_cap, in
   s.qth = o;   o = al(o + size_t(G) * 12 * 4, 128);
   s.scan = o;  o = al(o + size_t(kWarps + 1) * G * 4, 128);
   s.merge = o; o = al(o + size_t(kWarps) * kPartStride * 4, 128);
-  s.info = o;  o = al(o + size_t(G) * 8 * 4, 128);
+  s.info = o;  o = al(o + size_t(G) * 9 * 4, 128);
   s.misc = o;  o = al(o + 128, 128);
   s.total = o;
   return s;
+}
+
+// Bit 15 and bit 31 of w0, then of w1, as bits 0..3 (the sign bits of four packed
+// 16-bit lanes): a byte permute gathers the four high bytes, one multiply moves
+// their top bits to bits 28..31 without carries.
+__device__ __forceinline__ uint32_t lane_sign_bits(uint32_t w0, uint32_t w1) {
+  const uint32_t b = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+  return (b * 0x00204081u) >> 28;
 }
 
 // Exclusive prefix over the block (thread order) of G counters per thread; also
@@ -141,11 +156,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = a.cluster;
   const int rank = int(cluster.block_rank());
-  const SmemLayout lo = make_layout(G, a.keys_per_cta, a.list_cap, CS);
+  const int S = a.stages;
+  const SmemLayout lo = make_layout(G, a.keys_per_cta, a.list_cap, CS, S);
   uint8_t* ring = smem + lo.ring;
   float* part = reinterpret_cast<float*>(smem + lo.ring);           // [CS][G][kPartStride]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + lo.hist);    // [G][kBinStride]
+  uint32_t* coarse = reinterpret_cast<uint32_t*>(smem + lo.coarse);  // [CS][G][kCoarseRow]
+  uint32_t* fine = reinterpret_cast<uint32_t*>(smem + lo.fine);      // [CS][G][kFine]
   uint16_t* dist = reinterpret_cast<uint16_t*>(smem + lo.dist);    // [G][RS]
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + lo.list);    // [G][list_cap]
   float* qf = reinterpret_cast<float*>(smem + lo.qf);              // [G][128]
@@ -168,9 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 
   // ---- issue the code copies first: HBM traffic starts before anything else
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
+    for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
     fence_mbar_init();
-    for (int qi = 0; qi < min(nch, kStages); ++qi) {
+    for (int qi = 0; qi < min(nch, S); ++qi) {
       const int keys = min(kChunk, n - qi * kChunk);
       mbar_expect_tx(&mbar[qi], uint32_t(keys * kCodeBytes));
       bulk_g2s(ring + size_t(qi) * kChunk * kCodeBytes,
@@ -223,9 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
     }
     const int swz = (tid >> 2) & 1;   // conflict-free 2 x 16 B reads of a 32 B code
+    int slot = 0;
+    uint32_t parity = 0;
     for (int qi = 0; qi < nch; ++qi) {
-      const int slot = qi % kStages;
-      mbar_wait_bounded(&mbar[slot], uint32_t(qi / kStages) & 1u, a.err);
+      mbar_wait_bounded(&mbar[slot], parity, a.err);
       const int r = qi * kChunk + tid;
       if (r < n) {
         const uint4* src = reinterpret_cast<const uint4*>(
@@ -256,14 +275,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         }
       }
       __syncthreads();
-      if (tid == 0 && qi + kStages < nch) {
-        const int nx = qi + kStages;
+      if (tid == 0 && qi + S < nch) {
+        const int nx = qi + S;
         const int keys = min(kChunk, n - nx * kChunk);
         mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes));
         bulk_g2s(ring + size_t(slot) * kChunk * kCodeBytes,
                  codes + int64_t(nx) * kChunk * kCodeBytes, uint32_t(keys * kCodeBytes),
                  &mbar[slot]);
       }
+      if (++slot == S) { slot = 0; parity ^= 1u; }
     }
   }
 
@@ -293,39 +313,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     }
   }
 
-  cluster.sync();   // every CTA's cumulative histograms are complete and visible
+  __syncthreads();
+  // push this CTA's cumulative counts at the 30 coarse-chunk ends (+2 pad) into
+  // every peer: after the barrier the coarse level of the D* search is local
+  for (int i = tid; i < CS * G * (kCoarseRow / 4); i += kThreads) {
+    const int cc = i / (G * (kCoarseRow / 4));
+    const int g = (i / (kCoarseRow / 4)) % G;
+    const int q4 = i % (kCoarseRow / 4);
+    uint32_t v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * q4 + e;
+      v[e] = hist[g * kBinStride + min(kCoarse * j + kCoarse - 1, kNBins - 1)];
+    }
+    uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(coarse, cc) +
+                                          (size_t(rank) * G + g) * kCoarseRow) + q4;
+    *dst = make_uint4(v[0], v[1], v[2], v[3]);
+  }
 
-  // ---- resolve D*, the count selected in lower-ranked CTAs, and the ties taken
+  cluster.sync();   // cumulative histograms complete; coarse counts delivered
+
+  // ---- resolve D*, the count selected in lower-ranked CTAs, and the ties taken.
+  // Level 1 (local): the coarse chunk j* where the unit's cumulative count reaches
+  // k_eff.  Level 2: each peer's 20-bin window around chunk j* is pulled with
+  // 16-byte loads, then bins 13 j* - 1 .. 13 j* + 12 give D* exactly.
+  int* jst = info + G * 8;   // [G] coarse chunk per head
+  if (warp < G) {
+    const int g = warp;
+    uint32_t S1 = 0;
+    if (lane < kNCoarse) {
+      for (int cc = 0; cc < CS; ++cc) S1 += coarse[(cc * G + g) * kCoarseRow + lane];
+    }
+    const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < kNCoarse && S1 >= uint32_t(a.k_eff));
+    if (lane == 0) jst[g] = __ffs(hit1) - 1;   // exists: chunk 29 ends at bin 384, count L
+  }
+  __syncthreads();
+  for (int i = tid; i < CS * G * (kFine / 4); i += kThreads) {
+    const int cc = i / (G * (kFine / 4));
+    const int g = (i / (kFine / 4)) % G;
+    const int q4 = i % (kFine / 4);
+    const int lo_bin = min(max(0, kCoarse * jst[g] - 1) & ~3, kBinStride - kFine);
+    const uint4 v = *(reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, cc) +
+                                                      g * kBinStride + lo_bin) + q4);
+    *(reinterpret_cast<uint4*>(fine + (cc * G + g) * kFine) + q4) = v;
+  }
+  __syncthreads();
   if (warp < G) {
     const int g = warp;
     const uint32_t ke = uint32_t(a.k_eff);
-    // level 1: cumulative counts of the whole unit at the end of each coarse chunk;
-    // all peer loads are issued before any is summed
-    uint32_t S1 = 0;
-    if (lane < 30) {
-      const int bj = min(kCoarse * lane + kCoarse - 1, kNBins - 1);
-      uint32_t v[kMaxCluster];
-#pragma unroll
-      for (int cc = 0; cc < kMaxCluster; ++cc)
-        v[cc] = cc < CS ? cluster.map_shared_rank(hist, cc)[g * kBinStride + bj] : 0u;
-#pragma unroll
-      for (int cc = 0; cc < kMaxCluster; ++cc) S1 += v[cc];
-    }
-    const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < 30 && S1 >= ke);
-    const int jstar = __ffs(hit1) - 1;   // exists: the last chunk ends at bin 384, count L
-    // level 2: bins 13 j* - 1 .. 13 j* + 12 (lane l -> bin 13 j* - 1 + l)
+    const int jstar = jst[g];
+    const int lo_bin = min(max(0, kCoarse * jstar - 1) & ~3, kBinStride - kFine);
+    // level 2: lane l -> bin 13 j* - 1 + l
     const int d = kCoarse * jstar - 1 + lane;
     uint32_t S2 = 0, Sb = 0;
     if (lane < kCoarse + 1 && d >= 0) {
-      const int dd = min(d, kNBins - 1);
-      uint32_t v[kMaxCluster];
-#pragma unroll
-      for (int cc = 0; cc < kMaxCluster; ++cc)
-        v[cc] = cc < CS ? cluster.map_shared_rank(hist, cc)[g * kBinStride + dd] : 0u;
-#pragma unroll
-      for (int cc = 0; cc < kMaxCluster; ++cc) {
-        S2 += v[cc];
-        if (cc < rank) Sb += v[cc];
+      const int off = min(d, kNBins - 1) - lo_bin;
+      for (int cc = 0; cc < CS; ++cc) {
+        const uint32_t x = fine[(cc * G + g) * kFine + off];
+        S2 += x;
+        if (cc < rank) Sb += x;
       }
     }
     const uint32_t hit2 = __ballot_sync(0xffffffffu, lane >= 1 && lane < kCoarse + 1 && S2 >= ke);
@@ -372,22 +418,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       const int s0 = rb + tid * per;
       const int cntv = max(0, min(per, rb + nr - s0));
       uint32_t ltm[G], eqm[G], cnt[G], tot[G];
+      const uint32_t valid = cntv >= 32 ? 0xffffffffu : ((1u << cntv) - 1u);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        ltm[g] = eqm[g] = 0;
+        // packed compares, two distances per word: in each 16-bit lane
+        // (0x8000 + D*) - d keeps bit 15 iff d <= D*, (0x7fff + D*) - d iff d < D*
+        // (distances <= 384, so no lane borrows from its neighbour)
+        const uint32_t cle = (0x8000u + uint32_t(dstar[g])) * 0x10001u;
+        const uint32_t clt = cle - 0x10001u;
+        uint32_t lm = 0, em = 0;
         const uint16_t* row = dist + size_t(g) * RS + s0;
         for (int i8 = 0; i8 < cntv; i8 += 8) {
           const uint4 v = *reinterpret_cast<const uint4*>(row + i8);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int dv = int((w[j >> 1] >> (16 * (j & 1))) & 0xffffu);
-            const uint32_t bit = (i8 + j < cntv) ? (1u << (i8 + j)) : 0u;
-            if (dv < dstar[g]) ltm[g] |= bit;
-            if (dv == dstar[g]) eqm[g] |= bit;
+          const uint32_t l0 = lane_sign_bits(clt - v.x, clt - v.y);
+          const uint32_t l1 = lane_sign_bits(clt - v.z, clt - v.w);
+          const uint32_t e0 = lane_sign_bits(cle - v.x, cle - v.y) & ~l0;
+          const uint32_t e1 = lane_sign_bits(cle - v.z, cle - v.w) & ~l1;
+          lm |= (l0 | (l1 << 4)) << i8;
+          em |= (e0 | (e1 << 4)) << i8;
+        }
+        ltm[g] = lm & valid;
+        eqm[g] = em & valid;
+        cnt[g] = (uint32_t(__popc(ltm[g])) << 16) | uint32_t(__popc(eqm[g]));
+        // tokens below D* are selected whatever the tie rule decides: start pulling
+        // their K/V rows into L2 now, so the gather finds them there
+        if (a.attend) {
+          uint32_t m = ltm[g];
+          while (m) {
+            const int i = __ffs(m) - 1;
+            m &= m - 1u;
+            const int64_t row_off = (int64_t(unit) * a.Lmax + p0 + s0 + i) * kD;
+            prefetch_row_l2(static_cast<const T*>(a.k) + row_off);
+            prefetch_row_l2(static_cast<const T*>(a.v) + row_off);
           }
         }
-        cnt[g] = (uint32_t(__popc(ltm[g])) << 16) | uint32_t(__popc(eqm[g]));
       }
       block_exclusive_scan<G>(cnt, tot, scan, lane, warp);
 #pragma unroll
@@ -552,7 +616,11 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int sme
     if (R > 65535) continue;                       // positions in a CTA are 16-bit
     if (cs > 1 && (L + R - 1) / R < cs) continue;  // an all-empty tail CTA: use fewer
     const int list_cap = int(std::max<int64_t>(1, std::min<int64_t>(R, k_eff)));
-    const size_t smem = make_layout(G, int(R), list_cap, cs).total;
+    const int64_t nchunks = (R + kChunk - 1) / kChunk;
+    int stages = int(std::min<int64_t>(kMaxStages, std::max<int64_t>(1, nchunks)));
+    while (stages > 1 && make_layout(G, int(R), list_cap, cs, stages).total > size_t(smem_cap))
+      --stages;
+    const size_t smem = make_layout(G, int(R), list_cap, cs, stages).total;
     if (smem > size_t(smem_cap)) continue;
     int conc_clusters = sms / cs;
     if (query_device) conc_clusters = active_clusters(G, cs, smem);
@@ -569,6 +637,7 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int sme
       p.cluster = cs;
       p.keys_per_cta = R;
       p.list_cap = list_cap;
+      p.stages = stages;
       p.smem = smem;
       p.waves = int(waves);
     }
@@ -636,6 +705,7 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.cluster = p.cluster;
   a.keys_per_cta = int(p.keys_per_cta);
   a.list_cap = p.list_cap;
+  a.stages = p.stages;
   a.attend = out != nullptr ? 1 : 0;
   if (dt == ADAMAS_F32) return launch_t<float>(G, a, p, stream);
   return launch_t<__nv_bfloat16>(G, a, p, stream);

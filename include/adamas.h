@@ -142,6 +142,30 @@ adamas_status adamas_sparse_attention(const void* q, const void* k_cache, const 
                                       size_t ws_bytes, float* out, cudaStream_t stream);
 
 /*
+ * adamas_sparse_attention without a workspace, for callers that cannot allocate
+ * device memory: code running inside a memory allocator's own hooks, latency
+ * paths that must not call into the driver's allocator, or hosts whose memory
+ * pool owns every device allocation.  The paper has no counterpart to this entry
+ * point; it is an interface convenience.
+ *
+ * Same arguments, layouts and result as adamas_sparse_attention, minus the
+ * workspace.  Scratch (per-head counters and split partials, about 2.2 MB) is a
+ * fixed array inside the library that every GPU loading the library keeps until
+ * the process exits.  Limit: B * Hq <= 4096 (larger calls return
+ * ADAMAS_ERR_UNSUPPORTED); the split count is reduced so that B * Hq * splits
+ * <= 4096.  The FIRST call on each device looks up the array's device address
+ * and clears its counters, synchronizing the device; make that first call outside
+ * any stream capture.  All calls share the one array (each completed call leaves
+ * its counters at zero again), so calls that run concurrently on the GPU — from
+ * several streams or host threads — race and must be serialized by the caller.
+ */
+adamas_status adamas_sparse_attention_noalloc(const void* q, const void* k_cache,
+                                              const void* v_cache, adamas_dtype dt,
+                                              const int32_t* idx, int B, int Hq, int Hkv, int d,
+                                              int64_t Lmax, int k_eff, float* out,
+                                              cudaStream_t stream);
+
+/*
  * Launch plan of adamas_decode_step for these sizes on the current device (host
  * only, no launch): total CTAs, CTAs per thread-block cluster (one cluster per
  * (batch, kv head) pair), key positions per CTA, dynamic shared memory bytes per

@@ -52,6 +52,8 @@ _SIGNATURES = {
     "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "adamas_sparse_attention": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i, _c_i,
                                        _c_i64, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "adamas_sparse_attention_noalloc": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i,
+                                               _c_i, _c_i64, _c_i, _c_p, _c_p]),
     "adamas_decode_plan": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i64, _c_i,
                                   ctypes.POINTER(_c_i), ctypes.POINTER(_c_i),
                                   ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i)]),
@@ -231,7 +233,25 @@ def sparse_attention(q, k_cache, v_cache, idx, ws=None, out=None, stream=None):
     return out
 
 
+def sparse_attention_noalloc(q, k_cache, v_cache, idx, out=None, stream=None):
+    """adamas_sparse_attention without a workspace (library-held scratch; see
+    include/adamas.h for the size limit and the first-call set-up)."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if idx.dtype != torch.int32:
+        raise TypeError("idx must be int32")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _check(lib().adamas_sparse_attention_noalloc(_dev(q, "q"), _dev(k_cache, "k_cache"),
+                                                 _dev(v_cache, "v_cache"), _dtype_code(k_cache),
+                                                 _dev(idx, "idx"), B, Hq, Hkv, d, Lmax,
+                                                 idx.shape[-1], _dev(out, "out"),
+                                                 _stream(stream)),
+           "adamas_sparse_attention_noalloc")
+    return out
+
+
 __all__ = ["lib", "header_symbols", "status_string", "AdamasError", "encode_keys",
            "encode_queries", "decode_workspace_bytes", "decode_plan", "init_workspace",
            "decode_workspace", "check_workspace", "decode_step", "select_topk",
-           "sparse_attention_workspace", "sparse_attention"]
+           "sparse_attention_workspace", "sparse_attention", "sparse_attention_noalloc"]

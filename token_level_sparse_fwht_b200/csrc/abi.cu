@@ -181,4 +181,21 @@ adamas_status adamas_sparse_attention(const void* q, const void* k_cache, const 
                                            workspace, out, stream));
 }
 
+adamas_status adamas_sparse_attention_noalloc(const void* q, const void* k_cache,
+                                              const void* v_cache, adamas_dtype dt,
+                                              const int32_t* idx, int B, int Hq, int Hkv, int d,
+                                              int64_t Lmax, int k_eff, float* out,
+                                              cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !idx || !out || !good_dtype(dt)) return ADAMAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || k_eff <= 0 || Hq % Hkv)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(idx, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (!noalloc_fits(B, Hq)) return ADAMAS_ERR_UNSUPPORTED;   // B * Hq above the fixed scratch
+  return from_cuda(launch_sparse_attention_noalloc(q, k_cache, v_cache, dt, idx, B, Hq, Hkv, Lmax,
+                                                   k_eff, out, stream));
+}
+
 }  // extern "C"

@@ -387,6 +387,11 @@ cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, i
                                int64_t per, int64_t stride, int64_t off, float t,
                                cudaStream_t stream);
 size_t attention_workspace_bytes(int B, int Hq, int k_eff);
+bool noalloc_fits(int B, int Hq);
+cudaError_t launch_sparse_attention_noalloc(const void* q, const void* k, const void* v,
+                                            adamas_dtype dt, const int32_t* idx, int B,
+                                            int Hq, int Hkv, int64_t Lmax, int k_eff,
+                                            float* out, cudaStream_t stream);
 cudaError_t launch_sparse_attention(const void* q, const void* k, const void* v,
                                     adamas_dtype dt, const int32_t* idx, int B, int Hq,
                                     int Hkv, int64_t Lmax, int k_eff, void* ws, float* out,

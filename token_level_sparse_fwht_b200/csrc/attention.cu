@@ -10,6 +10,7 @@
 // (batch, head) — atomic counter in the workspace — merges the S partials and
 // resets its counter, so the workspace stays zero between calls.
 #include <algorithm>
+#include <mutex>
 
 #include "adamas_internal.cuh"
 
@@ -100,6 +101,86 @@ cudaError_t launch_sparse_attention(const void* q, const void* k, const void* v,
   float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align_up(heads * 4, 256));
   const float scale_log2 = float(1.4426950408889634 / 11.313708498984761);
   const unsigned grid = unsigned(heads * S);
+  if (dt == ADAMAS_BF16) {
+    sparse_attention_kernel<__nv_bfloat16><<<grid, kAttnThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), idx, Hq, Hkv, Lmax, k_eff, S, scale_log2, done,
+        part, out);
+  } else {
+    sparse_attention_kernel<float><<<grid, kAttnThreads, 0, stream>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        idx, Hq, Hkv, Lmax, k_eff, S, scale_log2, done, part, out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace adamas
+
+// ------------------------------------------------------------------------------
+// Allocation-free variant of adamas_sparse_attention.
+//
+// Some callers cannot hand the library a workspace: code that runs where
+// cudaMalloc is off limits (inside a custom allocator's own callbacks, in
+// real-time paths that must not block on the driver's allocator, or under a
+// framework whose memory pool owns every device allocation).  For them the split
+// partials and per-head counters live in this fixed, file-scope device array,
+// which every GPU that loads the library holds until the process exits.
+// ------------------------------------------------------------------------------
+namespace adamas {
+
+constexpr int kNoAllocMaxHeads = 4096;      // B * Hq per call
+constexpr int kNoAllocMaxPartials = 4096;   // B * Hq * splits per call
+constexpr size_t kNoAllocCounterBytes = 256 * ((kNoAllocMaxHeads * 4 + 255) / 256);
+constexpr size_t kNoAllocBytes =
+    kNoAllocCounterBytes + size_t(kNoAllocMaxPartials) * kPartStride * 4;
+
+// Host code may not use this name as a device address: the symbol's device
+// address is looked up once per device below and passed to the kernel.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+static std::mutex g_noalloc_mutex;
+static void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Once per device, with that device current: the scratch's device address, and
+// the counters cleared (each completed call returns them to zero by itself).
+static cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(p, 0, kNoAllocCounterBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+bool noalloc_fits(int B, int Hq) { return int64_t(B) * Hq <= kNoAllocMaxHeads; }
+
+cudaError_t launch_sparse_attention_noalloc(const void* q, const void* k, const void* v,
+                                            adamas_dtype dt, const int32_t* idx, int B,
+                                            int Hq, int Hkv, int64_t Lmax, int k_eff,
+                                            float* out, cudaStream_t stream) {
+  void* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  const int sms = current_device_sms(nullptr);
+  const int heads = B * Hq;
+  int S = attention_splits(B, Hq, k_eff, sms > 0 ? sms : 148);
+  S = std::max(1, std::min(S, kNoAllocMaxPartials / heads));
+  uint32_t* done = static_cast<uint32_t*>(scratch);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocCounterBytes);
+  const float scale_log2 = float(1.4426950408889634 / 11.313708498984761);
+  const unsigned grid = unsigned(heads) * unsigned(S);
   if (dt == ADAMAS_BF16) {
     sparse_attention_kernel<__nv_bfloat16><<<grid, kAttnThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),

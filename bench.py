@@ -131,6 +131,21 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings over all ranks (every rank calls it)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def aggregate_gbs(step_bytes: int, seconds_per_step: float, world: int) -> float:
+    """Whole-job effective GB/s under weak scaling: every rank runs its own step
+    (independent units, no collective on the data path); the job's time per step
+    is the slowest rank's."""
+    return step_bytes * world / seconds_per_step / 1e9
+
+
 # ------------------------------------------------------------- our arm
 def smi_id(dev) -> str:
     """nvidia-smi id of a torch device (UUID, so CUDA_VISIBLE_DEVICES does not matter)."""
@@ -276,11 +291,7 @@ def run_ours(args, rank, world, local):
     stream.synchronize()
     ms_e2e = f0.elapsed_time(f1)
 
-    # max over ranks
-    tt = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-    ms, ms_e2e = float(tt[0]), float(tt[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
     return dict(w=w, k=k, ms=ms, ms_e2e=ms_e2e, K=K, K2=K2, R=R, step_bytes=step_bytes,
                 clocks=clocks, plan=plan, use_graph=use_graph,
                 launches=K * launches_per_step,
@@ -400,8 +411,8 @@ def main():
     w, k = r["w"], r["k"]
     peak, peak_kind = peaks()
     per_step_s = r["ms"] / 1e3 / r["K"]
-    gbs_rank = r["step_bytes"] / per_step_s / 1e9
-    value = gbs_rank * world
+    gbs_rank = aggregate_gbs(r["step_bytes"], per_step_s, 1)
+    value = aggregate_gbs(r["step_bytes"], per_step_s, world)
     e2e_step_s = r["ms_e2e"] / 1e3 / r["K2"]
     key = f"config{args.config}_k{k}"
     line = {
@@ -430,7 +441,7 @@ def main():
                      "traffic": ncu_traffic(key),
                      "kernel": "decode_kernel (one launch per step)",
                      "peak_source": f"{peak_kind} hbm_gbs"},
-        "e2e": {"value": round(r["step_bytes"] * world / e2e_step_s / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(aggregate_gbs(r["step_bytes"], e2e_step_s, world), 2), "unit": "GB/s",
                 "us_per_step": round(e2e_step_s * 1e6, 3),
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],

@@ -269,13 +269,17 @@ def run_ours(args, rank, world, local):
     outs = torch.empty(out_host.shape, dtype=torch.float32, device=dev)
     K2 = max(3, min(K, 2000 // w.layers))
 
+    # per layer one C call: pinned q in, fused decode, fp32 out back to pinned host;
+    # the calls are bound to their buffers once, as a serving loop would
+    calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws, outs[li],
+                                    out_host[li], stream=stream)
+              for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
+
     def e2e_step(i):
-        q_dev.copy_(q_host, non_blocking=True)
         for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
             if append:
                 ad.encode_keys(kc, cd, L - append, append, t, stream=stream)
-            ad.decode_step(q_dev[li], kc, vc, cd, L, k, t, ws, out=outs[li], stream=stream)
-        out_host.copy_(outs, non_blocking=True)
+            calls[i % R][li]()
 
     with torch.cuda.stream(stream):
         for i in range(3):

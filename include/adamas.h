@@ -122,6 +122,24 @@ adamas_status adamas_decode_step(const void* q, const void* k_cache, const void*
                                  float* out, cudaStream_t stream);
 
 /*
+ * adamas_decode_step for a caller whose queries and outputs live in (preferably
+ * pinned) host memory: queues the copy q_host -> q_dev ([B][Hq][d] elements of
+ * `dt`), the decode step, and the copy out_dev -> out_host ([B][Hq][d] float32),
+ * all asynchronous on `stream` (synchronize before reading out_host).  q_dev and
+ * out_dev are caller-owned device staging buffers; the caches, codes, workspace
+ * and idx_out are as in adamas_decode_step.  When both host buffers are
+ * page-locked and mapped into the device's address space (cudaHostAlloc /
+ * cudaMallocHost memory on a unified-addressing system), the kernel reads q and
+ * writes the output through that mapping and the staging buffers are not used.
+ */
+adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const void* k_cache,
+                                      const void* v_cache, const uint8_t* codes, adamas_dtype dt,
+                                      int B, int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                      int k, float t, void* workspace, size_t ws_bytes,
+                                      int32_t* idx_out, float* out_dev, float* out_host,
+                                      cudaStream_t stream);
+
+/*
  * Stage entry point: distance scan + top-k from given query codes (no attention).
  * Same kernel as adamas_decode_step with the attention stages switched off.
  */

@@ -159,3 +159,43 @@ def test_decode_llama8b_128k_layers_sampled():
                               ocodes[(b, kv)], k, inp.t)
         del inp, codes, ws
         torch.cuda.empty_cache()
+
+
+def test_decode_step_host_buffers():
+    """adamas_decode_step_host (pinned q in, fp32 out back, one C call) returns what
+    adamas_decode_step returns for the same inputs, bit for bit."""
+    w = WORKLOADS[2].scaled(L=2500, Hq=16, Hkv=4)
+    inp = generate(w, "cpu")
+    kc = oracle_codes(inp.k_cache, inp.t)
+    kcache, vcache, codes = inp.k_cache.cuda(), inp.v_cache.cuda(), upload(kc)
+    ws = ad.decode_workspace(1, 16, 4, w.L, 128)
+    want = ad.decode_step(inp.q.cuda(), kcache, vcache, codes, w.L, 128, inp.t, ws)
+    q_host = inp.q.clone().pin_memory()
+    out_host = torch.zeros((1, 16, 128), dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(inp.q, device="cuda")
+    out_dev = torch.empty((1, 16, 128), dtype=torch.float32, device="cuda")
+    ad.decode_step_host(q_host, q_dev, kcache, vcache, codes, w.L, 128, inp.t, ws, out_dev,
+                        out_host)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, want.cpu())
+
+
+def test_prepared_decode_host_call():
+    """The prepared (buffer-bound) host call gives the same output as decode_step."""
+    w = WORKLOADS[2].scaled(L=1800, Hq=8, Hkv=2)
+    inp = generate(w, "cpu")
+    kcache, vcache = inp.k_cache.cuda(), inp.v_cache.cuda()
+    codes = upload(oracle_codes(inp.k_cache, inp.t))
+    ws = ad.decode_workspace(1, 8, 2, w.L, 64)
+    want = ad.decode_step(inp.q.cuda(), kcache, vcache, codes, w.L, 64, inp.t, ws).cpu()
+    q_host = inp.q.clone().pin_memory()
+    out_host = torch.zeros((1, 8, 128), dtype=torch.float32).pin_memory()
+    call = ad.PreparedDecodeHost(q_host, torch.empty_like(inp.q, device="cuda"), kcache, vcache,
+                                 codes, w.L, 64, inp.t, ws,
+                                 torch.empty((1, 8, 128), device="cuda"), out_host,
+                                 stream=torch.cuda.current_stream())
+    for _ in range(2):
+        out_host.zero_()
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(out_host, want)

@@ -47,6 +47,9 @@ _SIGNATURES = {
     "adamas_check_workspace": (_c_i, [_c_p, _c_sz, _c_p]),
     "adamas_decode_step": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i64,
                                   _c_i64, _c_i, _c_f, _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "adamas_decode_step_host": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i,
+                                       _c_i, _c_i64, _c_i64, _c_i, _c_f, _c_p, _c_sz, _c_p,
+                                       _c_p, _c_p, _c_p]),
     "adamas_select_topk": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i, _c_p,
                                   _c_sz, _c_p, _c_p]),
     "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
@@ -194,6 +197,54 @@ def decode_step(q, k_cache, v_cache, codes, L: int, k: int, t: float, ws, idx_ou
     return out
 
 
+def decode_step_host(q_host, q_dev, k_cache, v_cache, codes, L: int, k: int, t: float, ws,
+                     out_dev, out_host, idx_out=None, stream=None):
+    """decode_step with host-resident q and output: one C call queues the host->device
+    copy of q, the fused kernel and the device->host copy of out on `stream`."""
+    B, Hq, d = q_dev.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if q_host.is_cuda or out_host.is_cuda:
+        raise ValueError("q_host and out_host must be host tensors")
+    idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
+    _check(lib().adamas_decode_step_host(q_host.data_ptr(), _dev(q_dev, "q_dev"),
+                                         _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                         _dev(codes, "codes"), _dtype_code(k_cache), B, Hq, Hkv,
+                                         d, Lmax, L, k, float(t), _dev(ws, "workspace"),
+                                         ws.numel(), idx_ptr, _dev(out_dev, "out_dev"),
+                                         out_host.data_ptr(), _stream(stream)),
+           "adamas_decode_step_host")
+    return out_host
+
+
+class PreparedDecodeHost:
+    """A decode step bound to fixed buffers, for serving loops that reuse them every
+    step: all pointers and sizes are resolved once, so each call is one C call with
+    no per-call Python checks.  Same semantics as decode_step_host."""
+
+    def __init__(self, q_host, q_dev, k_cache, v_cache, codes, L: int, k: int, t: float, ws,
+                 out_dev, out_host, idx_out=None, stream=None):
+        B, Hq, d = q_dev.shape
+        _, Hkv, Lmax, _ = k_cache.shape
+        if q_host.is_cuda or out_host.is_cuda:
+            raise ValueError("q_host and out_host must be host tensors")
+        if tuple(q_host.shape) != (B, Hq, d) or tuple(out_host.shape) != (B, Hq, d):
+            raise ValueError("q_host / out_host shapes must be [B, Hq, d]")
+        self._keep = (q_host, q_dev, k_cache, v_cache, codes, ws, out_dev, out_host, idx_out)
+        self._fn = lib().adamas_decode_step_host
+        self._args = (
+            _c_p(q_host.data_ptr()), _c_p(_dev(q_dev, "q_dev")), _c_p(_dev(k_cache, "k_cache")),
+            _c_p(_dev(v_cache, "v_cache")), _c_p(_dev(codes, "codes")),
+            _c_i(_dtype_code(k_cache)), _c_i(B), _c_i(Hq), _c_i(Hkv), _c_i(d), _c_i64(Lmax),
+            _c_i64(L), _c_i(k), _c_f(t), _c_p(_dev(ws, "workspace")), _c_sz(ws.numel()),
+            _c_p(None if idx_out is None else _dev(idx_out, "idx_out")),
+            _c_p(_dev(out_dev, "out_dev")), _c_p(out_host.data_ptr()), _c_p(_stream(stream)))
+
+    def __call__(self):
+        status = self._fn(*self._args)
+        if status != OK:
+            raise AdamasError(status, "adamas_decode_step_host")
+
+
 def select_topk(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
     B, Hq, _ = qcodes.shape
     _, Hkv, Lmax, _ = codes.shape
@@ -252,6 +303,7 @@ def sparse_attention_noalloc(q, k_cache, v_cache, idx, out=None, stream=None):
 
 
 __all__ = ["lib", "header_symbols", "status_string", "AdamasError", "encode_keys",
+           "decode_step_host", "PreparedDecodeHost",
            "encode_queries", "decode_workspace_bytes", "decode_plan", "init_workspace",
            "decode_workspace", "check_workspace", "decode_step", "select_topk",
            "sparse_attention_workspace", "sparse_attention", "sparse_attention_noalloc"]

@@ -40,6 +40,19 @@ bool good_group(int Hq, int Hkv) {
 }
 adamas_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ADAMAS_OK : ADAMAS_ERR_CUDA; }
 
+// Device address of a page-locked, device-mapped host buffer; nullptr for any
+// other memory (pageable host memory, device memory, unknown pointers).
+template <typename P>
+P* mapped_device_pointer(P* host) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, host) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr) return nullptr;
+  return static_cast<P*>(attr.devicePointer);
+}
+
 // Shared checks of the decode / select entry points.
 adamas_status check_decode_sizes(int B, int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
                                  int k) {
@@ -141,6 +154,48 @@ adamas_status adamas_decode_step(const void* q, const void* k_cache, const void*
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv, Lmax, L,
                                  k, t, workspace, idx_out, out, p, stream));
+}
+
+adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const void* k_cache,
+                                      const void* v_cache, const uint8_t* codes, adamas_dtype dt,
+                                      int B, int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                      int k, float t, void* workspace, size_t ws_bytes,
+                                      int32_t* idx_out, float* out_dev, float* out_host,
+                                      cudaStream_t stream) {
+  if (!q_host || !out_host) return ADAMAS_ERR_INVALID_ARG;
+  // everything else is checked by adamas_decode_step before the copy is queued
+  if (!q_dev || !k_cache || !v_cache || !codes || !workspace || !out_dev || !good_dtype(dt) ||
+      !good_t(t))
+    return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(q_dev, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(codes, 16) || !aligned(out_dev, 16) || !aligned(workspace, 256) ||
+      (idx_out && !aligned(idx_out, 4)))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  // Page-locked host buffers are mapped into the device's address space: then the
+  // kernel reads q from, and writes out to, host memory itself (no copy engines,
+  // no extra stream operations).  Otherwise the copies go through q_dev / out_dev.
+  const void* qh_dev = mapped_device_pointer(q_host);
+  void* oh_dev = mapped_device_pointer(out_host);
+  if (qh_dev && oh_dev && aligned(qh_dev, 16) && aligned(oh_dev, 16)) {
+    return from_cuda(launch_decode(qh_dev, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
+                                   Lmax, L, k, t, workspace, idx_out, static_cast<float*>(oh_dev),
+                                   p, stream));
+  }
+  const size_t elem = dt == ADAMAS_F32 ? 4 : 2;
+  const size_t qbytes = size_t(B) * Hq * kD * elem;
+  const size_t obytes = size_t(B) * Hq * kD * sizeof(float);
+  if (cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return ADAMAS_ERR_CUDA;
+  const adamas_status r = from_cuda(launch_decode(q_dev, nullptr, k_cache, v_cache, codes, dt, B,
+                                                  Hq, Hkv, Lmax, L, k, t, workspace, idx_out,
+                                                  out_dev, p, stream));
+  if (r != ADAMAS_OK) return r;
+  return from_cuda(cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, stream));
 }
 
 adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, int B, int Hq,

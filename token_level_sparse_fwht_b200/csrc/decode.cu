@@ -40,7 +40,7 @@ namespace adamas {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = kThreads;  // keys per bulk copy (16 KiB of codes), one per thread
-constexpr int kMaxStages = 4;    // bulk-copy ring depth (runtime: 2..4, as shared memory allows)
+constexpr int kMaxStages = 8;    // bulk-copy ring depth (runtime: 1..8, as shared memory allows)
 constexpr int kMaxCluster = 16;  // non-portable cluster size limit
 constexpr int kCoarse = 13;      // bins per coarse chunk of the D* search (30 chunks)
 constexpr int kNCoarse = 30;     // coarse chunks (30 x 13 >= 385 bins)
@@ -93,7 +93,7 @@ __host__ __device__ inline SmemLayout make_layout(int G, int R, int list_cap, in
   s.qf = o;    o = al(o + size_t(G) * kD * 4, 128);
   s.qc = o;    o = al(o + size_t(G) * kCodeBytes, 128);
   s.qth = o;   o = al(o + size_t(G) * 12 * 4, 128);
-  s.scan = o;  o = al(o + size_t(kWarps + 1) * G * 4, 128);
+  s.scan = o;  o = al(o + size_t(2) * kWarps * G * 4, 128);
   s.merge = o; o = al(o + size_t(kWarps) * kPartStride * 4, 128);
   s.info = o;  o = al(o + size_t(G) * 9 * 4, 128);
   s.misc = o;  o = al(o + 128, 128);
@@ -109,11 +109,16 @@ __device__ __forceinline__ uint32_t lane_sign_bits(uint32_t w0, uint32_t w1) {
   return (b * 0x00204081u) >> 28;
 }
 
-// Exclusive prefix over the block (thread order) of G counters per thread; also
-// returns the block totals.  scan holds (kWarps + 1) x G words.
+// Exclusive prefix over the block (thread order) of G counters per thread, and the
+// block totals, with one barrier: warp totals go to shared memory and every thread
+// adds up the totals of the warps before it.  `scan` holds two buffers of
+// kWarps x G words used alternately (by `parity`), so a call never overwrites
+// totals that a slower warp may still be reading from the previous call.
 template <int G>
 __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t (&total)[G],
-                                                     uint32_t* scan, int lane, int warp) {
+                                                     uint32_t* scan, int parity, int lane,
+                                                     int warp) {
+  uint32_t* buf = scan + parity * kWarps * G;
   uint32_t inc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -124,30 +129,26 @@ __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t 
       if (lane >= o) x += y;
     }
     inc[g] = x;
-    if (lane == 31) scan[warp * G + g] = x;
+    if (lane == 31) buf[warp * G + g] = x;
   }
   __syncthreads();
-  if (warp == 0) {
+  uint32_t before[G], tot[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) before[g] = tot[g] = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const uint32_t own = lane < kWarps ? scan[lane * G + g] : 0u;
-      uint32_t x = own;
-#pragma unroll
-      for (int o = 1; o < kWarps; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (lane < kWarps) scan[lane * G + g] = x - own;
-      if (lane == kWarps - 1) scan[kWarps * G + g] = x;
+      const uint32_t x = buf[w * G + g];
+      tot[g] += x;
+      before[g] += w < warp ? x : 0u;
     }
   }
-  __syncthreads();
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    v[g] = scan[warp * G + g] + inc[g] - v[g];
-    total[g] = scan[kWarps * G + g];
+    v[g] = before[g] + inc[g] - v[g];
+    total[g] = tot[g];
   }
-  __syncthreads();
 }
 
 template <int G, typename T>
@@ -184,8 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   const int nch = (n + kChunk - 1) / kChunk;
   const uint8_t* codes = a.codes + (int64_t(unit) * a.Lmax + p0) * kCodeBytes;
 
-  // ---- issue the code copies first: HBM traffic starts before anything else
-  if (tid == 0) {
+  // ---- issue the code copies first: HBM traffic starts before anything else.  The
+  // last warp issues them, so the warps that encode the queries are not delayed.
+  if (tid == kThreads - 32) {
     for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
     fence_mbar_init();
     for (int qi = 0; qi < min(nch, S); ++qi) {
@@ -274,8 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           }
         }
       }
-      __syncthreads();
-      if (tid == 0 && qi + S < nch) {
+      // a slot is refilled only when the CTA's keys need more chunks than the ring
+      // holds; otherwise every chunk has its own slot and warps run ahead freely
+      if (nch > S) __syncthreads();
+      if (tid == kThreads - 32 && qi + S < nch) {
         const int nx = qi + S;
         const int keys = min(kChunk, n - nx * kChunk);
         mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes));
@@ -286,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       if (++slot == S) { slot = 0; parity ^= 1u; }
     }
   }
+  __syncthreads();   // every key's distances and histogram counts are in
 
   // ---- histograms -> inclusive cumulative histograms, in place (warp per head)
   if (warp < G) {
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     uint32_t carry_lt[G], carry_eq[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) carry_lt[g] = carry_eq[g] = 0;
-    for (int rb = 0; rb < n; rb += kRound) {
+    for (int rb = 0, parity = 0; rb < n; rb += kRound, parity ^= 1) {
       const int nr = min(kRound, n - rb);
       const int per = (((nr + kThreads - 1) / kThreads) + 7) & ~7;   // multiple of 8, <= 32
       const int s0 = rb + tid * per;
@@ -453,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           }
         }
       }
-      block_exclusive_scan<G>(cnt, tot, scan, lane, warp);
+      block_exclusive_scan<G>(cnt, tot, scan, parity, lane, warp);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int lt_b = int(carry_lt[g] + (cnt[g] >> 16));

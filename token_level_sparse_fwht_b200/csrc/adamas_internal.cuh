@@ -212,7 +212,7 @@ __device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane
 // becomes (odd, even) = ([c >= 3], [c >= 1]).
 __device__ __forceinline__ uint32_t therm13(uint32_t w) {
   const uint32_t d = (w >> 1) & ~w & 0x55555555u;      // h & ~l, at the even bit
-  return w ^ d ^ (d << 1);
+  return w ^ (d * 3u);   // d has even bits only: d * 3 = d | d << 1 (on the FMA pipe)
 }
 // [c >= 2] of two words, the first at even bits, the second at odd bits.
 __device__ __forceinline__ uint32_t therm2(uint32_t w0, uint32_t w1) {
@@ -249,20 +249,28 @@ __device__ __forceinline__ uint32_t therm_dist(const Therm& k, const Therm& q) {
 // at a time (sum word = a^b^c, carry word = majority(a,b,c), both single LOP3s),
 // so 8 popcounts replace 12.  POPC issues at a quarter of the integer-logic rate on
 // sm_100, so this moves work from the saturated popcount pipe to the logic pipe.
-__device__ __forceinline__ uint32_t therm_dist_csa(const Therm& k, const Therm& q) {
+__device__ __forceinline__ uint32_t therm_dist_csa(const Therm& k, const Therm& q,
+                                                   uint32_t one) {
   uint32_t x[12];
 #pragma unroll
   for (int i = 0; i < 8; ++i) x[i] = k.a[i] ^ q.a[i];
 #pragma unroll
   for (int i = 0; i < 4; ++i) x[8 + i] = k.b[i] ^ q.b[i];
+  // The sums run as integer multiply-adds with a multiplier the compiler cannot
+  // fold (one == 1 at run time), which keeps them on the FMA pipe and leaves the
+  // integer-logic pipe, the scan's bottleneck, to the XOR / carry-save work.
   uint32_t ones = 0, twos = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t a = x[3 * j], b = x[3 * j + 1], c = x[3 * j + 2];
-    ones += __popc(a ^ b ^ c);
-    twos += __popc((a & b) | (c & (a | b)));
+    asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(ones) : "r"(uint32_t(__popc(a ^ b ^ c))), "r"(one));
+    asm("mad.lo.u32 %0, %1, %2, %0;"
+        : "+r"(twos)
+        : "r"(uint32_t(__popc((a & b) | (c & (a | b))))), "r"(one));
   }
-  return ones + 2u * twos;
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(twos), "r"(one + one), "r"(ones));
+  return r;
 }
 
 // ---------------------------------------------------------- warp utilities
@@ -285,18 +293,19 @@ struct SoftmaxState {
 
 // Gathers up to `n` rows (positions from `pos_of(j)` for j = j0, j0+step, ...)
 // and folds them into `st`.  K/V row r of this (batch, kv head) starts at
-// base + r * kD.  Four rows are in flight per warp per batch.
+// base + r * kD.  kRows rows (K and V) are in flight per warp per batch.
 template <typename T, typename PosFn>
 __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
                                             const T* __restrict__ vbase, int n, int j0,
                                             int step, PosFn pos_of, const float q[4],
                                             float scale_log2, int lane, SoftmaxState& st) {
   using R = Raw4<T>;
-  for (int j = j0; j < n; j += 4 * step) {
-    typename R::type kr[4], vr[4];
-    bool valid[4];
+  constexpr int kRows = 8;
+  for (int j = j0; j < n; j += kRows * step) {
+    typename R::type kr[kRows], vr[kRows];
+    bool valid[kRows];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kRows; ++u) {
       const int jj = j + u * step;
       valid[u] = jj < n;
       if (valid[u]) {
@@ -305,9 +314,9 @@ __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
         vr[u] = R::load(vbase + pos * kD, lane);
       }
     }
-    float s[4];
+    float s[kRows];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kRows; ++u) {
       float kv[4];
       if (valid[u]) {
         R::decode(kr[u], kv);
@@ -319,11 +328,11 @@ __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+      for (int u = 0; u < kRows; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
     }
     float mx = st.m;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kRows; ++u) {
       s[u] = valid[u] ? s[u] * scale_log2 : -INFINITY;
       mx = fmaxf(mx, s[u]);
     }
@@ -332,7 +341,7 @@ __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
 #pragma unroll
     for (int r = 0; r < 4; ++r) st.acc[r] *= corr;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kRows; ++u) {
       if (valid[u]) {
         const float p = exp2f(s[u] - mx);
         float vv[4];

@@ -243,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
     }
     const int swz = (tid >> 2) & 1;   // conflict-free 2 x 16 B reads of a 32 B code
+    const uint32_t one = uint32_t(a.keys_per_cta > 0);   // 1, opaque to the compiler
     int slot = 0;
     uint32_t parity = 0;
     for (int qi = 0; qi < nch; ++qi) {
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           }
 #pragma unroll
           for (int g = 0; g < GR; ++g) {
-            const uint32_t dd = therm_dist_csa(kt, qreg[g]);
+            const uint32_t dd = therm_dist_csa(kt, qreg[g], one);
             dist[size_t(g0 + g) * RS + r] = static_cast<uint16_t>(dd);
             atomicAdd(&hist[(g0 + g) * kBinStride + dd], 1u);
           }
@@ -316,24 +317,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       run += loc[i];
       if (bin < kNBins) row[bin] = run;
     }
-  }
-
-  __syncthreads();
-  // push this CTA's cumulative counts at the 30 coarse-chunk ends (+2 pad) into
-  // every peer: after the barrier the coarse level of the D* search is local
-  for (int i = tid; i < CS * G * (kCoarseRow / 4); i += kThreads) {
-    const int cc = i / (G * (kCoarseRow / 4));
-    const int g = (i / (kCoarseRow / 4)) % G;
-    const int q4 = i % (kCoarseRow / 4);
-    uint32_t v[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = 4 * q4 + e;
-      v[e] = hist[g * kBinStride + min(kCoarse * j + kCoarse - 1, kNBins - 1)];
+    // push this CTA's cumulative counts at the 30 coarse-chunk ends (+2 pad) into
+    // every peer, so the coarse level of the D* search reads local memory after
+    // the barrier.  Lane j now holds the count at the end of chunk j (lanes 29..31:
+    // the total); four lanes are gathered per 16-byte remote store.
+    const int g = warp;
+    const uint32_t c0 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 0);
+    const uint32_t c1 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 1);
+    const uint32_t c2 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 2);
+    const uint32_t c3 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 3);
+    if (lane < kCoarseRow / 4) {
+      for (int cc = 0; cc < CS; ++cc) {
+        uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(coarse, cc) +
+                                              (size_t(rank) * G + g) * kCoarseRow) + lane;
+        *dst = make_uint4(c0, c1, c2, c3);
+      }
     }
-    uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(coarse, cc) +
-                                          (size_t(rank) * G + g) * kCoarseRow) + q4;
-    *dst = make_uint4(v[0], v[1], v[2], v[3]);
   }
 
   cluster.sync();   // cumulative histograms complete; coarse counts delivered
@@ -424,26 +423,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       const int cntv = max(0, min(per, rb + nr - s0));
       uint32_t ltm[G], eqm[G], cnt[G], tot[G];
       const uint32_t valid = cntv >= 32 ? 0xffffffffu : ((1u << cntv) - 1u);
+      // packed compares, two distances per word: in each 16-bit lane
+      // (0x8000 + D*) - d keeps bit 15 iff d <= D*, (0x7fff + D*) - d iff d < D*
+      // (distances <= 384, so no lane borrows from its neighbour).  All G heads'
+      // loads of a group of 8 positions are issued before any compare.
+      uint32_t cle[G], clt[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        // packed compares, two distances per word: in each 16-bit lane
-        // (0x8000 + D*) - d keeps bit 15 iff d <= D*, (0x7fff + D*) - d iff d < D*
-        // (distances <= 384, so no lane borrows from its neighbour)
-        const uint32_t cle = (0x8000u + uint32_t(dstar[g])) * 0x10001u;
-        const uint32_t clt = cle - 0x10001u;
-        uint32_t lm = 0, em = 0;
-        const uint16_t* row = dist + size_t(g) * RS + s0;
-        for (int i8 = 0; i8 < cntv; i8 += 8) {
-          const uint4 v = *reinterpret_cast<const uint4*>(row + i8);
-          const uint32_t l0 = lane_sign_bits(clt - v.x, clt - v.y);
-          const uint32_t l1 = lane_sign_bits(clt - v.z, clt - v.w);
-          const uint32_t e0 = lane_sign_bits(cle - v.x, cle - v.y) & ~l0;
-          const uint32_t e1 = lane_sign_bits(cle - v.z, cle - v.w) & ~l1;
-          lm |= (l0 | (l1 << 4)) << i8;
-          em |= (e0 | (e1 << 4)) << i8;
+        cle[g] = (0x8000u + uint32_t(dstar[g])) * 0x10001u;
+        clt[g] = cle[g] - 0x10001u;
+        ltm[g] = eqm[g] = 0;
+      }
+      for (int i8 = 0; i8 < cntv; i8 += 8) {
+        uint4 v[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          v[g] = *reinterpret_cast<const uint4*>(dist + size_t(g) * RS + s0 + i8);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const uint32_t l0 = lane_sign_bits(clt[g] - v[g].x, clt[g] - v[g].y);
+          const uint32_t l1 = lane_sign_bits(clt[g] - v[g].z, clt[g] - v[g].w);
+          const uint32_t e0 = lane_sign_bits(cle[g] - v[g].x, cle[g] - v[g].y) & ~l0;
+          const uint32_t e1 = lane_sign_bits(cle[g] - v[g].z, cle[g] - v[g].w) & ~l1;
+          ltm[g] |= (l0 | (l1 << 4)) << i8;
+          eqm[g] |= (e0 | (e1 << 4)) << i8;
         }
-        ltm[g] = lm & valid;
-        eqm[g] = em & valid;
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        ltm[g] &= valid;
+        eqm[g] &= valid;
         cnt[g] = (uint32_t(__popc(ltm[g])) << 16) | uint32_t(__popc(eqm[g]));
         // tokens below D* are selected whatever the tie rule decides: start pulling
         // their K/V rows into L2 now, so the gather finds them there

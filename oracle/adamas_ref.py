@@ -206,3 +206,44 @@ def decode_head(q_vec, K_rows, V_rows, k, t, key_codes_rows=None, query_code=Non
     dist = manhattan(unpack_codes(query_code), unpack_codes(key_codes_rows))
     sel = select_topk(dist, k)
     return sel, sparse_attention(q_vec, K_rows, V_rows, sel), dist
+
+
+# ------------------------------------------------ shared GQA selection variant
+def decode_step_shared(q: np.ndarray, K: np.ndarray, V: np.ndarray, k: int, t: float,
+                       key_codes: np.ndarray | None = None,
+                       query_codes: np.ndarray | None = None):
+    """Decode step with one selection per kv head, shared by its G query heads.
+
+    A variant the pages leave open (the v2 abstract selects top-k positions but
+    says nothing about grouped-query attention): the score of key j for kv head
+    h_kv is the SUM over the group's query heads of their Manhattan distances to
+    key j's code; the first min(k, L) positions under (sum asc, position asc) are
+    gathered once and every query head of the group attends over them.
+    Returns (idx [B, Hkv, k_eff] ascending, out [B, Hq, d] float64).
+    """
+    q = np.asarray(q)
+    B, Hq, d = q.shape
+    _, Hkv, L, _ = K.shape
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    if key_codes is None:
+        key_codes = encode(K, t)
+    if query_codes is None:
+        query_codes = encode(q, t)
+    ck = unpack_codes(np.asarray(key_codes)[:, :, :L])
+    cq = unpack_codes(np.asarray(query_codes))
+    k_eff = min(int(k), L)
+    idx = np.zeros((B, Hkv, k_eff), dtype=np.int64)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    for b in range(B):
+        for kvh in range(Hkv):
+            score = np.zeros(L, dtype=np.int64)
+            for g in range(G):
+                score += manhattan(cq[b, kvh * G + g], ck[b, kvh])
+            sel = select_topk(score, k)
+            idx[b, kvh] = sel
+            for g in range(G):
+                h = kvh * G + g
+                out[b, h] = sparse_attention(q[b, h], K[b, kvh, :L], V[b, kvh, :L], sel)
+    return idx, out

@@ -242,6 +242,65 @@ def check_planted_recall_single_head():
     assert planted <= set(idx[0, 0].tolist())
 
 
+# ---------------------------------------------------- shared GQA selection
+def check_shared_g1_is_per_head():
+    """With one query head per kv head, shared selection IS per-head selection."""
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((2, 3, 128))
+    K = rng.standard_normal((2, 3, 90, 128))
+    V = rng.standard_normal((2, 3, 90, 128))
+    i1, o1 = ref.decode_step(q, K, V, k=17, t=0.4)
+    i2, o2 = ref.decode_step_shared(q, K, V, k=17, t=0.4)
+    assert np.array_equal(i1, i2) and np.allclose(o1, o2, atol=1e-12)
+
+
+def check_shared_bruteforce():
+    """Pure-Python sum of per-head Manhattan distances, full sort by (sum, position),
+    and torch dense attention over the selected rows for every head of the group."""
+    rng = np.random.default_rng(37)
+    B, Hq, Hkv, L, k, t = 1, 4, 2, 40, 9, 0.3
+    G = Hq // Hkv
+    q = rng.standard_normal((B, Hq, 128))
+    K = rng.standard_normal((B, Hkv, L, 128))
+    V = rng.standard_normal((B, Hkv, L, 128))
+    idx, out = ref.decode_step_shared(q, K, V, k=k, t=t)
+    cq = ref.unpack_codes(ref.encode(q, t))
+    ck = ref.unpack_codes(ref.encode(K, t))
+    for kvh in range(Hkv):
+        score = []
+        for j in range(L):
+            s = 0
+            for g in range(G):
+                for i in range(128):
+                    s += abs(int(cq[0, kvh * G + g, i]) - int(ck[0, kvh, j, i]))
+            score.append(s)
+        want = sorted(sorted(range(L), key=lambda j: (score[j], j))[:k])
+        assert list(idx[0, kvh]) == want, (kvh, list(idx[0, kvh]), want)
+        for g in range(G):
+            h = kvh * G + g
+            dense = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[0, h])[None, None, None, :],
+                torch.from_numpy(K[0, kvh, want])[None, None],
+                torch.from_numpy(V[0, kvh, want])[None, None])[0, 0, 0].numpy()
+            assert np.allclose(out[0, h], dense, atol=1e-12)
+
+
+def check_shared_identical_heads():
+    """If every query head of a group is the same vector, the summed score is G times
+    each head's distance, so the shared selection equals each head's own."""
+    rng = np.random.default_rng(41)
+    q0 = rng.standard_normal((1, 2, 128))
+    q = np.repeat(q0, 4, axis=1)                  # Hq = 8, Hkv = 2, G = 4
+    K = rng.standard_normal((1, 2, 120, 128))
+    V = rng.standard_normal((1, 2, 120, 128))
+    i_head, o_head = ref.decode_step(q, K, V, k=20, t=0.5)
+    i_sh, o_sh = ref.decode_step_shared(q, K, V, k=20, t=0.5)
+    for kvh in range(2):
+        for g in range(4):
+            assert np.array_equal(i_sh[0, kvh], i_head[0, kvh * 4 + g])
+    assert np.allclose(o_sh, o_head, atol=1e-12)
+
+
 ALL_CHECKS = [
     check_hadamard_matches_scipy, check_hadamard_orthogonal,
     check_rotate_involution_and_dot, check_rotate_closed_forms, check_bucket_golden,
@@ -249,4 +308,5 @@ ALL_CHECKS = [
     check_simhash_reduction, check_topk_bruteforce, check_topk_special,
     check_attention_dense, check_attention_budget1, check_decode_dense_limit,
     check_gqa_and_planted, check_planted_recall_single_head,
+    check_shared_g1_is_per_head, check_shared_bruteforce, check_shared_identical_heads,
 ]

@@ -11,7 +11,7 @@ from pins import ALL_CHECKS
 
 _orig = {name: getattr(ref, name) for name in (
     "sylvester_hadamard", "hadamard_rotate", "bucketize", "pack_codes", "unpack_codes",
-    "manhattan", "select_topk", "sparse_attention", "decode_step")}
+    "manhattan", "select_topk", "sparse_attention", "decode_step", "decode_step_shared")}
 
 
 def _h_or(n=128):                      # popcount(i | j) instead of i & j
@@ -103,6 +103,17 @@ def _decode_mod_gqa(q, K, V, k, t, key_codes=None, query_codes=None):
     return idx[:, back], out[:, back]
 
 
+def _shared_first_head_only(q, K, V, k, t, key_codes=None, query_codes=None):
+    # shared selection scored by the group's first query head alone
+    B, Hq, d = q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    qq = np.repeat(np.asarray(q)[:, ::G], G, axis=1)
+    idx, _ = _orig["decode_step_shared"](qq, K, V, k, t)
+    _, out = _orig["decode_step_shared"](q, K, V, k, t)
+    return idx, out
+
+
 MUTATIONS = {
     "hadamard_or": ("sylvester_hadamard", _h_or),
     "rotate_unscaled": ("hadamard_rotate", _rotate_unscaled),
@@ -117,6 +128,7 @@ MUTATIONS = {
     "attention_noscale": ("sparse_attention", _attn_noscale),
     "attention_k_as_v": ("sparse_attention", _attn_uses_k),
     "decode_gqa_modulo": ("decode_step", _decode_mod_gqa),
+    "shared_first_head_only": ("decode_step_shared", _shared_first_head_only),
 }
 
 
@@ -130,6 +142,6 @@ def test_mutation_is_caught(name, monkeypatch):
             check()
         except AssertionError:
             failed.append(check.__name__)
-        except Exception:               # a crash also counts as caught
-            failed.append(check.__name__ + "!")
+        except Exception as e:          # a crash in a pin is a test bug, not a catch
+            raise AssertionError(f"{check.__name__} crashed under {name}: {e!r}")
     assert failed, f"mutation {name} passed every pin"

@@ -1,12 +1,14 @@
 """Benchmark of the Adamas decode step on B200: µs per step and effective HBM GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--budget 128]
-                    [--impl ours|reference]
+                    [--shared] [--impl ours|reference]
 
 Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32 query / 8 kv heads,
 d = 128, context 32768, bf16 K/V with 4 outlier channels, budget 128.  A "step" is
 one adamas_decode_step (query encode, distance scan, top-k, gather attention,
-combine: one cooperative kernel launch).
+combine: one thread-block-cluster kernel launch).  --shared times the variant with
+one selection per kv head shared by its query heads (adamas_decode_step_shared);
+its algorithmic bytes count the selected K/V rows once per kv head.
 
 Timing: inputs resident in HBM; R independent replicas of codes + K + V are
 rotated so the working set of consecutive steps exceeds 2x L2 (no cache reuse
@@ -175,7 +177,9 @@ def run_ours(args, rank, world, local):
         del inp
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     append = w.append
-    step_bytes = w.algorithmic_bytes(k) * w.layers
+    shared = args.shared
+    decode = ad.decode_step_shared if shared else ad.decode_step
+    step_bytes = w.algorithmic_bytes(k, shared) * w.layers
     if append:
         step_bytes += w.B * w.Hkv * append * (128 * w.elem_bytes + 32)
     R = args.replicas or replicas_for_l2(step_bytes, l2, 2.0)
@@ -185,15 +189,15 @@ def run_ours(args, rank, world, local):
     ws = ad.decode_workspace(w.B, w.Hq, w.Hkv, L, k, dev)
     out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
-    plan = ad.decode_plan(w.B, w.Hq, w.Hkv, L, k)
+    plan = (ad.decode_plan_shared if shared else ad.decode_plan)(w.B, w.Hq, w.Hkv, L, k)
     launches_per_step = w.layers * (2 if append else 1)
 
     def step(i, s, q_override=None):
         for (q, kc, vc, cd) in sets[i % R]:
             if append:
                 ad.encode_keys(kc, cd, L - append, append, t, stream=s)
-            ad.decode_step(q if q_override is None else q_override, kc, vc, cd, L, k, t, ws,
-                           out=out, stream=s)
+            decode(q if q_override is None else q_override, kc, vc, cd, L, k, t, ws, out=out,
+                   stream=s)
 
     # eager warm-up (also loads the kernels and sets their attributes)
     with torch.cuda.stream(stream):
@@ -272,7 +276,7 @@ def run_ours(args, rank, world, local):
     # per layer one C call: pinned q in, fused decode, fp32 out back to pinned host;
     # the calls are bound to their buffers once, as a serving loop would
     calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws, outs[li],
-                                    out_host[li], stream=stream)
+                                    out_host[li], stream=stream, shared=shared)
               for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
 
     def e2e_step(i):
@@ -314,21 +318,23 @@ def oracle_inputs(w, seed_device="cpu"):
     return inp.t, q, K, V, oracle
 
 
-def cpu_baseline(w, k, budget_s=12.0):
+def cpu_baseline(w, k, budget_s=12.0, shared=False):
     """The oracle's full decode step (all heads) on the host, repeated for about
     budget_s seconds: effective GB/s over the same algorithmic bytes."""
     t, q, K, V, oracle = oracle_inputs(w)
     kc = oracle.encode(K, t)        # key codes are cache state, built before timing
+    fn = oracle.decode_step_shared if shared else oracle.decode_step
     n = 0
     t0 = time.perf_counter()
     while True:
-        oracle.decode_step(q, K, V, k, t, key_codes=kc)
+        fn(q, K, V, k, t, key_codes=kc)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 50:
             break
     per_step = el / n
-    return {"value": w.algorithmic_bytes(k) / per_step / 1e9, "unit": "GB/s", "cores": 1,
+    return {"value": w.algorithmic_bytes(k, shared) / per_step / 1e9, "unit": "GB/s",
+            "cores": 1,
             "kind": "oracle",
             "sample": f"{n} full decode steps of the same workload (all {w.B * w.Hq} heads), "
                       f"{per_step * 1e3:.0f} ms each, numpy float64, single thread"}
@@ -396,6 +402,8 @@ def main():
     ap.add_argument("--replicas", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shared", action="store_true",
+                    help="shared GQA selection (one top-k per kv head)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.budget is None:
@@ -418,7 +426,7 @@ def main():
     gbs_rank = aggregate_gbs(r["step_bytes"], per_step_s, 1)
     value = aggregate_gbs(r["step_bytes"], per_step_s, world)
     e2e_step_s = r["ms_e2e"] / 1e3 / r["K2"]
-    key = f"config{args.config}_k{k}"
+    key = f"config{args.config}_k{k}" + ("_shared" if args.shared else "")
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -436,6 +444,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128, "L": w.L,
                    "k": k, "algorithmic_bytes_per_step": r["step_bytes"],
+                   "selection": "shared per kv head" if args.shared else "per query head",
                    "replicas": r["R"], "l2": "rotated replicas, working set >= 2x L2",
                    "layers": w.layers, "append_tokens": w.append,
                    "graph": r["use_graph"], "ctas": r["plan"]["ctas"],
@@ -452,7 +461,7 @@ def main():
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, k)
+        line["cpu_baseline"] = cpu_baseline(w, k, shared=args.shared)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

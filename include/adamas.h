@@ -59,7 +59,8 @@ typedef enum {
   ADAMAS_ERR_INVALID_ARG = 1,
   ADAMAS_ERR_UNSUPPORTED = 2,
   ADAMAS_ERR_CUDA = 3,
-  ADAMAS_ERR_TIMEOUT = 4
+  ADAMAS_ERR_TIMEOUT = 4,
+  ADAMAS_ERR_INTERNAL = 5
 } adamas_status;
 
 typedef enum { ADAMAS_F32 = 0, ADAMAS_BF16 = 1 } adamas_dtype;
@@ -100,8 +101,10 @@ adamas_status adamas_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stre
 /*
  * SYNCHRONIZES `stream`, then reads the device error word of a decode workspace.
  * Returns ADAMAS_ERR_TIMEOUT if a kernel gave up a bounded wait (completion of a
- * bulk copy into shared memory) since the workspace was initialised, else
- * ADAMAS_OK (or ADAMAS_ERR_CUDA if the stream reported an error).
+ * bulk copy into shared memory) since the workspace was initialised,
+ * ADAMAS_ERR_INTERNAL if the top-k bookkeeping of a kernel found no k-th distance
+ * (inconsistent counts: a bug, never expected), else ADAMAS_OK (or ADAMAS_ERR_CUDA
+ * if the stream reported an error).
  */
 adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -147,6 +150,39 @@ adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, in
                                  int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
                                  size_t ws_bytes, int32_t* idx_out, cudaStream_t stream);
 
+/*
+ * Shared GQA selection (a variant the Adamas pages leave open: the v2 abstract of
+ * "Adamas: Hadamard Sparse Attention for Efficient Long-Context Inference" picks
+ * top-k positions per query but does not treat grouped-query attention).  For
+ * each (batch, kv head) the score of key j is the SUM over the G = Hq / Hkv query
+ * heads of the group of their Manhattan code distances to key j (0 .. 384 G); the
+ * first min(k, L) positions under (score ascending, position ascending) are
+ * selected ONCE, and every query head of the group attends over that one set, so
+ * each selected K/V row is read once per group instead of once per query head.
+ * Arguments, layouts, ownership and errors are those of adamas_decode_step, except
+ * idx_out, which receives [B][Hkv][k_eff] positions, ascending.
+ */
+adamas_status adamas_decode_step_shared(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
+                                        void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                        float* out, cudaStream_t stream);
+
+/* adamas_decode_step_host for the shared selection (idx_out [B][Hkv][k_eff]). */
+adamas_status adamas_decode_step_shared_host(const void* q_host, void* q_dev,
+                                             const void* k_cache, const void* v_cache,
+                                             const uint8_t* codes, adamas_dtype dt, int B,
+                                             int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                             int k, float t, void* workspace, size_t ws_bytes,
+                                             int32_t* idx_out, float* out_dev, float* out_host,
+                                             cudaStream_t stream);
+
+/* adamas_select_topk for the shared selection: idx_out [B][Hkv][k_eff]. */
+adamas_status adamas_select_topk_shared(const uint8_t* qcodes, const uint8_t* codes, int B,
+                                        int Hq, int Hkv, int64_t Lmax, int64_t L, int k,
+                                        void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                        cudaStream_t stream);
+
 /* Workspace of adamas_sparse_attention, in bytes (zero-filled once, self-cleaning). */
 size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff);
 
@@ -191,6 +227,11 @@ adamas_status adamas_sparse_attention_noalloc(const void* q, const void* k_cache
  */
 adamas_status adamas_decode_plan(int B, int Hq, int Hkv, int d, int64_t L, int k, int* ctas,
                                  int* cluster, int64_t* tokens_per_cta, int* smem_bytes);
+
+/* adamas_decode_plan of adamas_decode_step_shared / adamas_select_topk_shared. */
+adamas_status adamas_decode_plan_shared(int B, int Hq, int Hkv, int d, int64_t L, int k,
+                                        int* ctas, int* cluster, int64_t* tokens_per_cta,
+                                        int* smem_bytes);
 
 #ifdef __cplusplus
 }

@@ -112,3 +112,32 @@ def test_workspace_sizes_and_plan():
         assert q["smem_bytes"] <= 232448
     tiny = ad.decode_plan(3, 4, 4, 1, 1)                # L = 1: one key per unit
     assert tiny["cluster"] == 1 and tiny["tokens_per_cta"] == 1 and tiny["ctas"] == 12
+
+
+def test_shared_entry_points_reject_and_plan():
+    f = ad.lib().adamas_decode_step_shared
+    args = [A, A, A, A, BF16, 1, 32, 8, 128, 4096, 4096, 128, 1.0, A, 1 << 30, None, A, None]
+    bad = list(args); bad[0] = None
+    assert f(*bad) == ERR_INVALID_ARG
+    bad = list(args); bad[6] = 24                         # G = 3
+    assert f(*bad) == ERR_UNSUPPORTED
+    bad = list(args); bad[10] = 5000                      # L > Lmax
+    assert f(*bad) == ERR_INVALID_ARG
+    bad = list(args); bad[14] = 16                        # workspace too small
+    assert f(*bad) == ERR_INVALID_ARG
+    s = ad.lib().adamas_select_topk_shared
+    assert s(None, A, 1, 32, 8, 100, 100, 10, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    assert s(A, A, 1, 48, 8, 100, 100, 10, A, 1 << 30, A, None) == ERR_UNSUPPORTED
+    h = ad.lib().adamas_decode_step_shared_host
+    assert h(None, A, A, A, A, BF16, 1, 32, 8, 128, 4096, 4096, 128, 1.0, A, 1 << 30, None, A,
+             A, None) == ERR_INVALID_ARG
+    # shared selection needs wider histograms (384 G + 1 bins) and, for G > 1, a
+    # per-warp merge buffer for several heads: plans still fit the B200 cap
+    for args in [(1, 32, 8, 32768, 128), (4, 32, 8, 131072, 1024), (1, 64, 8, 65536, 256),
+                 (2, 16, 8, 10000, 100), (1, 8, 8, 4096, 64), (1, 2, 1, 70000, 50)]:
+        q = ad.decode_plan_shared(*args)
+        B, Hq, Hkv, L, k = args
+        assert q["ctas"] == B * Hkv * q["cluster"] and 1 <= q["cluster"] <= 16
+        assert q["tokens_per_cta"] * q["cluster"] >= L and q["tokens_per_cta"] <= 65535
+        assert q["smem_bytes"] <= 232448
+    assert ad.decode_plan_shared(1, 32, 8, 32768, 128)["cluster"] == 16

@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libadamas.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "adamas.h")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_INTERNAL = range(6)
 F32, BF16 = 0, 1
 HEAD_DIM = 128
 
@@ -52,6 +52,14 @@ _SIGNATURES = {
                                        _c_p, _c_p, _c_p]),
     "adamas_select_topk": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i, _c_p,
                                   _c_sz, _c_p, _c_p]),
+    "adamas_decode_step_shared": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                         _c_i64, _c_i64, _c_i, _c_f, _c_p, _c_sz, _c_p, _c_p,
+                                         _c_p]),
+    "adamas_decode_step_shared_host": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i,
+                                              _c_i, _c_i, _c_i64, _c_i64, _c_i, _c_f, _c_p,
+                                              _c_sz, _c_p, _c_p, _c_p, _c_p]),
+    "adamas_select_topk_shared": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i,
+                                         _c_p, _c_sz, _c_p, _c_p]),
     "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "adamas_sparse_attention": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i, _c_i,
                                        _c_i64, _c_i, _c_p, _c_sz, _c_p, _c_p]),
@@ -60,6 +68,9 @@ _SIGNATURES = {
     "adamas_decode_plan": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i64, _c_i,
                                   ctypes.POINTER(_c_i), ctypes.POINTER(_c_i),
                                   ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i)]),
+    "adamas_decode_plan_shared": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i64, _c_i,
+                                         ctypes.POINTER(_c_i), ctypes.POINTER(_c_i),
+                                         ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i)]),
 }
 
 
@@ -150,14 +161,24 @@ def decode_workspace_bytes(B: int, Hq: int, Hkv: int, L: int, k: int) -> int:
     return int(n)
 
 
-def decode_plan(B: int, Hq: int, Hkv: int, L: int, k: int) -> dict:
+def _plan(name: str, B: int, Hq: int, Hkv: int, L: int, k: int) -> dict:
     ctas, cluster, smem = _c_i(), _c_i(), _c_i()
     rng = _c_i64()
-    _check(lib().adamas_decode_plan(B, Hq, Hkv, HEAD_DIM, L, k, ctypes.byref(ctas),
-                                    ctypes.byref(cluster), ctypes.byref(rng),
-                                    ctypes.byref(smem)), "adamas_decode_plan")
+    _check(getattr(lib(), name)(B, Hq, Hkv, HEAD_DIM, L, k, ctypes.byref(ctas),
+                                ctypes.byref(cluster), ctypes.byref(rng), ctypes.byref(smem)),
+           name)
     return {"ctas": ctas.value, "cluster": cluster.value, "tokens_per_cta": rng.value,
             "smem_bytes": smem.value}
+
+
+def decode_plan(B: int, Hq: int, Hkv: int, L: int, k: int) -> dict:
+    """Launch plan of decode_step (host only): ctas, cluster, tokens_per_cta, smem_bytes."""
+    return _plan("adamas_decode_plan", B, Hq, Hkv, L, k)
+
+
+def decode_plan_shared(B: int, Hq: int, Hkv: int, L: int, k: int) -> dict:
+    """Launch plan of decode_step_shared / select_topk_shared."""
+    return _plan("adamas_decode_plan_shared", B, Hq, Hkv, L, k)
 
 
 def init_workspace(ws: torch.Tensor, stream=None):
@@ -180,49 +201,75 @@ def check_workspace(ws: torch.Tensor, stream=None):
 
 
 # -------------------------------------------------------------- decode step
-def decode_step(q, k_cache, v_cache, codes, L: int, k: int, t: float, ws, idx_out=None,
-                out=None, stream=None):
-    """One decode step (fused kernel).  Returns out [B,Hq,128] fp32 (and fills idx_out
-    [B,Hq,min(k,L)] int32 if given)."""
+def _decode(name, q, k_cache, v_cache, codes, L, k, t, ws, idx_out, out, stream):
     B, Hq, d = q.shape
     _, Hkv, Lmax, _ = k_cache.shape
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
     idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
-    _check(lib().adamas_decode_step(_dev(q, "q"), _dev(k_cache, "k_cache"),
-                                    _dev(v_cache, "v_cache"), _dev(codes, "codes"),
-                                    _dtype_code(k_cache), B, Hq, Hkv, d, Lmax, L, k, float(t),
-                                    _dev(ws, "workspace"), ws.numel(), idx_ptr,
-                                    _dev(out, "out"), _stream(stream)), "adamas_decode_step")
+    _check(getattr(lib(), name)(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                _dev(codes, "codes"), _dtype_code(k_cache), B, Hq, Hkv, d, Lmax,
+                                L, k, float(t), _dev(ws, "workspace"), ws.numel(), idx_ptr,
+                                _dev(out, "out"), _stream(stream)), name)
     return out
+
+
+def decode_step(q, k_cache, v_cache, codes, L: int, k: int, t: float, ws, idx_out=None,
+                out=None, stream=None):
+    """One decode step (fused kernel).  Returns out [B,Hq,128] fp32 (and fills idx_out
+    [B,Hq,min(k,L)] int32 if given)."""
+    return _decode("adamas_decode_step", q, k_cache, v_cache, codes, L, k, t, ws, idx_out, out,
+                   stream)
+
+
+def decode_step_shared(q, k_cache, v_cache, codes, L: int, k: int, t: float, ws, idx_out=None,
+                       out=None, stream=None):
+    """Decode step with one selection per kv head shared by its query heads (scores
+    summed over the group).  Returns out [B,Hq,128] fp32; idx_out, if given, is
+    [B,Hkv,min(k,L)] int32."""
+    return _decode("adamas_decode_step_shared", q, k_cache, v_cache, codes, L, k, t, ws,
+                   idx_out, out, stream)
 
 
 def decode_step_host(q_host, q_dev, k_cache, v_cache, codes, L: int, k: int, t: float, ws,
                      out_dev, out_host, idx_out=None, stream=None):
     """decode_step with host-resident q and output: one C call queues the host->device
     copy of q, the fused kernel and the device->host copy of out on `stream`."""
+    return _decode_host("adamas_decode_step_host", q_host, q_dev, k_cache, v_cache, codes, L,
+                        k, t, ws, out_dev, out_host, idx_out, stream)
+
+
+def decode_step_shared_host(q_host, q_dev, k_cache, v_cache, codes, L: int, k: int, t: float,
+                            ws, out_dev, out_host, idx_out=None, stream=None):
+    """decode_step_host for the shared selection (idx_out [B,Hkv,min(k,L)])."""
+    return _decode_host("adamas_decode_step_shared_host", q_host, q_dev, k_cache, v_cache,
+                        codes, L, k, t, ws, out_dev, out_host, idx_out, stream)
+
+
+def _decode_host(name, q_host, q_dev, k_cache, v_cache, codes, L, k, t, ws, out_dev, out_host,
+                 idx_out, stream):
     B, Hq, d = q_dev.shape
     _, Hkv, Lmax, _ = k_cache.shape
     if q_host.is_cuda or out_host.is_cuda:
         raise ValueError("q_host and out_host must be host tensors")
     idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
-    _check(lib().adamas_decode_step_host(q_host.data_ptr(), _dev(q_dev, "q_dev"),
-                                         _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-                                         _dev(codes, "codes"), _dtype_code(k_cache), B, Hq, Hkv,
-                                         d, Lmax, L, k, float(t), _dev(ws, "workspace"),
-                                         ws.numel(), idx_ptr, _dev(out_dev, "out_dev"),
-                                         out_host.data_ptr(), _stream(stream)),
-           "adamas_decode_step_host")
+    _check(getattr(lib(), name)(q_host.data_ptr(), _dev(q_dev, "q_dev"),
+                                _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                _dev(codes, "codes"), _dtype_code(k_cache), B, Hq, Hkv, d, Lmax,
+                                L, k, float(t), _dev(ws, "workspace"), ws.numel(), idx_ptr,
+                                _dev(out_dev, "out_dev"), out_host.data_ptr(), _stream(stream)),
+           name)
     return out_host
 
 
 class PreparedDecodeHost:
     """A decode step bound to fixed buffers, for serving loops that reuse them every
     step: all pointers and sizes are resolved once, so each call is one C call with
-    no per-call Python checks.  Same semantics as decode_step_host."""
+    no per-call Python checks.  Same semantics as decode_step_host (shared=True:
+    decode_step_shared_host)."""
 
     def __init__(self, q_host, q_dev, k_cache, v_cache, codes, L: int, k: int, t: float, ws,
-                 out_dev, out_host, idx_out=None, stream=None):
+                 out_dev, out_host, idx_out=None, stream=None, shared: bool = False):
         B, Hq, d = q_dev.shape
         _, Hkv, Lmax, _ = k_cache.shape
         if q_host.is_cuda or out_host.is_cuda:
@@ -230,7 +277,8 @@ class PreparedDecodeHost:
         if tuple(q_host.shape) != (B, Hq, d) or tuple(out_host.shape) != (B, Hq, d):
             raise ValueError("q_host / out_host shapes must be [B, Hq, d]")
         self._keep = (q_host, q_dev, k_cache, v_cache, codes, ws, out_dev, out_host, idx_out)
-        self._fn = lib().adamas_decode_step_host
+        self._name = "adamas_decode_step_shared_host" if shared else "adamas_decode_step_host"
+        self._fn = getattr(lib(), self._name)
         self._args = (
             _c_p(q_host.data_ptr()), _c_p(_dev(q_dev, "q_dev")), _c_p(_dev(k_cache, "k_cache")),
             _c_p(_dev(v_cache, "v_cache")), _c_p(_dev(codes, "codes")),
@@ -242,20 +290,30 @@ class PreparedDecodeHost:
     def __call__(self):
         status = self._fn(*self._args)
         if status != OK:
-            raise AdamasError(status, "adamas_decode_step_host")
+            raise AdamasError(status, self._name)
 
 
-def select_topk(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
+def _select(name, rows_per_batch, qcodes, codes, L, k, ws, idx_out, stream):
     B, Hq, _ = qcodes.shape
     _, Hkv, Lmax, _ = codes.shape
     k_eff = min(k, L)
     if idx_out is None:
-        idx_out = torch.empty((B, Hq, k_eff), dtype=torch.int32, device=qcodes.device)
-    _check(lib().adamas_select_topk(_dev(qcodes, "qcodes"), _dev(codes, "codes"), B, Hq, Hkv,
-                                    Lmax, L, k, _dev(ws, "workspace"), ws.numel(),
-                                    _dev(idx_out, "idx_out"), _stream(stream)),
-           "adamas_select_topk")
+        rows = Hq if rows_per_batch == "Hq" else Hkv
+        idx_out = torch.empty((B, rows, k_eff), dtype=torch.int32, device=qcodes.device)
+    _check(getattr(lib(), name)(_dev(qcodes, "qcodes"), _dev(codes, "codes"), B, Hq, Hkv, Lmax,
+                                L, k, _dev(ws, "workspace"), ws.numel(),
+                                _dev(idx_out, "idx_out"), _stream(stream)), name)
     return idx_out
+
+
+def select_topk(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
+    """Distance scan + per-head top-k from query codes: idx [B,Hq,min(k,L)] int32."""
+    return _select("adamas_select_topk", "Hq", qcodes, codes, L, k, ws, idx_out, stream)
+
+
+def select_topk_shared(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
+    """Shared selection from query codes: idx [B,Hkv,min(k,L)] int32."""
+    return _select("adamas_select_topk_shared", "Hkv", qcodes, codes, L, k, ws, idx_out, stream)
 
 
 def sparse_attention_workspace(B: int, Hq: int, k_eff: int, device="cuda", stream=None):

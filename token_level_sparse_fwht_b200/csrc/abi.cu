@@ -76,6 +76,7 @@ const char* adamas_status_string(adamas_status s) {
     case ADAMAS_ERR_UNSUPPORTED: return "unsupported configuration";
     case ADAMAS_ERR_CUDA: return "CUDA error";
     case ADAMAS_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case ADAMAS_ERR_INTERNAL: return "inconsistent top-k counts on the device";
   }
   return "unknown status";
 }
@@ -121,15 +122,22 @@ adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream
   if (cudaMemcpyAsync(&word, p, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return ADAMAS_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
-  return word ? ADAMAS_ERR_TIMEOUT : ADAMAS_OK;
+  if (word & (kErrBarrier | kErrCopy)) return ADAMAS_ERR_TIMEOUT;
+  return word ? ADAMAS_ERR_INTERNAL : ADAMAS_OK;
 }
 
-adamas_status adamas_decode_plan(int B, int Hq, int Hkv, int d, int64_t L, int k, int* ctas,
-                                 int* cluster, int64_t* tokens_per_cta, int* smem_bytes) {
+}  // extern "C"
+
+namespace {
+
+// The per-head and the shared-selection flavours of the decode / select entry
+// points differ only in the kernel instance and in the idx_out shape.
+adamas_status plan_common(bool shared, int B, int Hq, int Hkv, int d, int64_t L, int k,
+                          int* ctas, int* cluster, int64_t* tokens_per_cta, int* smem_bytes) {
   const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, L, L, k);
   if (s != ADAMAS_OK) return s;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
   if (ctas) *ctas = p.grid;
   if (cluster) *cluster = p.cluster;
   if (tokens_per_cta) *tokens_per_cta = p.keys_per_cta;
@@ -137,11 +145,11 @@ adamas_status adamas_decode_plan(int B, int Hq, int Hkv, int d, int64_t L, int k
   return ADAMAS_OK;
 }
 
-adamas_status adamas_decode_step(const void* q, const void* k_cache, const void* v_cache,
-                                 const uint8_t* codes, adamas_dtype dt, int B, int Hq,
-                                 int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
-                                 void* workspace, size_t ws_bytes, int32_t* idx_out,
-                                 float* out, cudaStream_t stream) {
+adamas_status decode_common(bool shared, const void* q, const void* k_cache,
+                            const void* v_cache, const uint8_t* codes, adamas_dtype dt, int B,
+                            int Hq, int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
+                            void* workspace, size_t ws_bytes, int32_t* idx_out, float* out,
+                            cudaStream_t stream) {
   if (!q || !k_cache || !v_cache || !codes || !workspace || !out) return ADAMAS_ERR_INVALID_ARG;
   if (!good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
   const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
@@ -150,20 +158,20 @@ adamas_status adamas_decode_step(const void* q, const void* k_cache, const void*
       !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv, Lmax, L,
-                                 k, t, workspace, idx_out, out, p, stream));
+                                 k, t, workspace, idx_out, out, shared, p, stream));
 }
 
-adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const void* k_cache,
-                                      const void* v_cache, const uint8_t* codes, adamas_dtype dt,
-                                      int B, int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
-                                      int k, float t, void* workspace, size_t ws_bytes,
-                                      int32_t* idx_out, float* out_dev, float* out_host,
-                                      cudaStream_t stream) {
+adamas_status decode_host_common(bool shared, const void* q_host, void* q_dev,
+                                 const void* k_cache, const void* v_cache, const uint8_t* codes,
+                                 adamas_dtype dt, int B, int Hq, int Hkv, int d, int64_t Lmax,
+                                 int64_t L, int k, float t, void* workspace, size_t ws_bytes,
+                                 int32_t* idx_out, float* out_dev, float* out_host,
+                                 cudaStream_t stream) {
   if (!q_host || !out_host) return ADAMAS_ERR_INVALID_ARG;
-  // everything else is checked by adamas_decode_step before the copy is queued
+  // everything else is checked here before the copy is queued
   if (!q_dev || !k_cache || !v_cache || !codes || !workspace || !out_dev || !good_dtype(dt) ||
       !good_t(t))
     return ADAMAS_ERR_INVALID_ARG;
@@ -174,7 +182,7 @@ adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const voi
       (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   // Page-locked host buffers are mapped into the device's address space: then the
   // kernel reads q from, and writes out to, host memory itself (no copy engines,
@@ -184,7 +192,7 @@ adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const voi
   if (qh_dev && oh_dev && aligned(qh_dev, 16) && aligned(oh_dev, 16)) {
     return from_cuda(launch_decode(qh_dev, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
                                    Lmax, L, k, t, workspace, idx_out, static_cast<float*>(oh_dev),
-                                   p, stream));
+                                   shared, p, stream));
   }
   const size_t elem = dt == ADAMAS_F32 ? 4 : 2;
   const size_t qbytes = size_t(B) * Hq * kD * elem;
@@ -193,14 +201,14 @@ adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const voi
     return ADAMAS_ERR_CUDA;
   const adamas_status r = from_cuda(launch_decode(q_dev, nullptr, k_cache, v_cache, codes, dt, B,
                                                   Hq, Hkv, Lmax, L, k, t, workspace, idx_out,
-                                                  out_dev, p, stream));
+                                                  out_dev, shared, p, stream));
   if (r != ADAMAS_OK) return r;
   return from_cuda(cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, stream));
 }
 
-adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, int B, int Hq,
-                                 int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
-                                 size_t ws_bytes, int32_t* idx_out, cudaStream_t stream) {
+adamas_status select_common(bool shared, const uint8_t* qcodes, const uint8_t* codes, int B,
+                            int Hq, int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
+                            size_t ws_bytes, int32_t* idx_out, cudaStream_t stream) {
   if (!qcodes || !codes || !workspace || !idx_out) return ADAMAS_ERR_INVALID_ARG;
   const adamas_status s = check_decode_sizes(B, Hq, Hkv, kD, Lmax, L, k);
   if (s != ADAMAS_OK) return s;
@@ -208,10 +216,82 @@ adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, in
       !aligned(idx_out, 4))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(nullptr, qcodes, nullptr, nullptr, codes, ADAMAS_BF16, B, Hq,
-                                 Hkv, Lmax, L, k, 0.0f, workspace, idx_out, nullptr, p, stream));
+                                 Hkv, Lmax, L, k, 0.0f, workspace, idx_out, nullptr, shared, p,
+                                 stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+adamas_status adamas_decode_plan(int B, int Hq, int Hkv, int d, int64_t L, int k, int* ctas,
+                                 int* cluster, int64_t* tokens_per_cta, int* smem_bytes) {
+  return plan_common(false, B, Hq, Hkv, d, L, k, ctas, cluster, tokens_per_cta, smem_bytes);
+}
+
+adamas_status adamas_decode_plan_shared(int B, int Hq, int Hkv, int d, int64_t L, int k,
+                                        int* ctas, int* cluster, int64_t* tokens_per_cta,
+                                        int* smem_bytes) {
+  return plan_common(true, B, Hq, Hkv, d, L, k, ctas, cluster, tokens_per_cta, smem_bytes);
+}
+
+adamas_status adamas_decode_step(const void* q, const void* k_cache, const void* v_cache,
+                                 const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                 int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
+                                 void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                 float* out, cudaStream_t stream) {
+  return decode_common(false, q, k_cache, v_cache, codes, dt, B, Hq, Hkv, d, Lmax, L, k, t,
+                       workspace, ws_bytes, idx_out, out, stream);
+}
+
+adamas_status adamas_decode_step_shared(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, int64_t L, int k, float t,
+                                        void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                        float* out, cudaStream_t stream) {
+  return decode_common(true, q, k_cache, v_cache, codes, dt, B, Hq, Hkv, d, Lmax, L, k, t,
+                       workspace, ws_bytes, idx_out, out, stream);
+}
+
+adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const void* k_cache,
+                                      const void* v_cache, const uint8_t* codes, adamas_dtype dt,
+                                      int B, int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                      int k, float t, void* workspace, size_t ws_bytes,
+                                      int32_t* idx_out, float* out_dev, float* out_host,
+                                      cudaStream_t stream) {
+  return decode_host_common(false, q_host, q_dev, k_cache, v_cache, codes, dt, B, Hq, Hkv, d,
+                            Lmax, L, k, t, workspace, ws_bytes, idx_out, out_dev, out_host,
+                            stream);
+}
+
+adamas_status adamas_decode_step_shared_host(const void* q_host, void* q_dev,
+                                             const void* k_cache, const void* v_cache,
+                                             const uint8_t* codes, adamas_dtype dt, int B,
+                                             int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                             int k, float t, void* workspace, size_t ws_bytes,
+                                             int32_t* idx_out, float* out_dev, float* out_host,
+                                             cudaStream_t stream) {
+  return decode_host_common(true, q_host, q_dev, k_cache, v_cache, codes, dt, B, Hq, Hkv, d,
+                            Lmax, L, k, t, workspace, ws_bytes, idx_out, out_dev, out_host,
+                            stream);
+}
+
+adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, int B, int Hq,
+                                 int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
+                                 size_t ws_bytes, int32_t* idx_out, cudaStream_t stream) {
+  return select_common(false, qcodes, codes, B, Hq, Hkv, Lmax, L, k, workspace, ws_bytes,
+                       idx_out, stream);
+}
+
+adamas_status adamas_select_topk_shared(const uint8_t* qcodes, const uint8_t* codes, int B,
+                                        int Hq, int Hkv, int64_t Lmax, int64_t L, int k,
+                                        void* workspace, size_t ws_bytes, int32_t* idx_out,
+                                        cudaStream_t stream) {
+  return select_common(true, qcodes, codes, B, Hq, Hkv, Lmax, L, k, workspace, ws_bytes,
+                       idx_out, stream);
 }
 
 size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff) {

@@ -18,6 +18,7 @@ constexpr int kPartStride = 132;        // m, l, 2 pad, acc[128] (floats)
 // error word bits (workspace header)
 constexpr uint32_t kErrBarrier = 1u;
 constexpr uint32_t kErrCopy = 2u;
+constexpr uint32_t kErrSelect = 4u;   // top-k bookkeeping found no k-th distance
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
 
 // ----------------------------------------------------------------- PTX helpers
@@ -355,6 +356,78 @@ __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
   }
 }
 
+// attend_rows for a group of GM query heads that share one selection: each K/V row
+// is loaded once and scored against all GM queries (q[g][4] is lane's slice of
+// query g); st[g] is head g's state.  kRows rows are in flight per warp.
+template <typename T, int GM, int kRows, typename PosFn>
+__device__ __forceinline__ void attend_rows_group(const T* __restrict__ kbase,
+                                                  const T* __restrict__ vbase, int n, int j0,
+                                                  int step, PosFn pos_of,
+                                                  const float (&q)[GM][4], float scale_log2,
+                                                  int lane, SoftmaxState (&st)[GM]) {
+  using R = Raw4<T>;
+  for (int j = j0; j < n; j += kRows * step) {
+    typename R::type kr[kRows], vr[kRows];
+    bool valid[kRows];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      const int jj = j + u * step;
+      valid[u] = jj < n;
+      if (valid[u]) {
+        const int64_t pos = pos_of(jj);
+        kr[u] = R::load(kbase + pos * kD, lane);
+        vr[u] = R::load(vbase + pos * kD, lane);
+      }
+    }
+    float s[GM][kRows];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      float kv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid[u]) R::decode(kr[u], kv);
+#pragma unroll
+      for (int g = 0; g < GM; ++g)
+        s[g][u] = q[g][0] * kv[0] + q[g][1] * kv[1] + q[g][2] * kv[2] + q[g][3] * kv[3];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int g = 0; g < GM; ++g) {
+#pragma unroll
+        for (int u = 0; u < kRows; ++u) s[g][u] += __shfl_xor_sync(0xffffffffu, s[g][u], o);
+      }
+    }
+    float vv[kRows][4];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      vv[u][0] = vv[u][1] = vv[u][2] = vv[u][3] = 0.f;
+      if (valid[u]) R::decode(vr[u], vv[u]);
+    }
+#pragma unroll
+    for (int g = 0; g < GM; ++g) {
+      float mx = st[g].m;
+#pragma unroll
+      for (int u = 0; u < kRows; ++u) {
+        s[g][u] = valid[u] ? s[g][u] * scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[g][u]);
+      }
+      const float corr = exp2f(st[g].m - mx);   // st.m = -inf -> 0
+      st[g].l *= corr;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) st[g].acc[r] *= corr;
+#pragma unroll
+      for (int u = 0; u < kRows; ++u) {
+        if (valid[u]) {
+          const float p = exp2f(s[g][u] - mx);
+          st[g].l += p;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) st[g].acc[r] = fmaf(p, vv[u][r], st[g].acc[r]);
+        }
+      }
+      st[g].m = mx;
+    }
+  }
+}
+
 // Merge two softmax partials (m, l, acc) into (M, Lsum, A) accumulators.
 __device__ __forceinline__ void merge_into(float m, float l, float a, float& M, float& Ls,
                                            float& A) {
@@ -385,13 +458,14 @@ struct Plan {
   int stages;            // bulk-copy ring depth
   size_t smem;           // dynamic shared memory bytes
 };
-bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, Plan& p);
+bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
+                                    Plan& p);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k);
 size_t decode_workspace_error_offset();
 cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
                           int64_t Lmax, int64_t L, int kk, float t, void* ws, int32_t* idx_out,
-                          float* out, const Plan& p, cudaStream_t stream);
+                          float* out, bool shared, const Plan& p, cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
                                cudaStream_t stream);

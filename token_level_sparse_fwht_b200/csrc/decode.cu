@@ -42,10 +42,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = kThreads;  // keys per bulk copy (16 KiB of codes), one per thread
 constexpr int kMaxStages = 8;    // bulk-copy ring depth (runtime: 1..8, as shared memory allows)
 constexpr int kMaxCluster = 16;  // non-portable cluster size limit
-constexpr int kCoarse = 13;      // bins per coarse chunk of the D* search (30 chunks)
-constexpr int kNCoarse = 30;     // coarse chunks (30 x 13 >= 385 bins)
+constexpr int kNCoarse = 30;     // coarse chunks of the D* search (30 x chunk >= bins)
 constexpr int kCoarseRow = 32;   // coarse counts per (CTA, head), padded to 128 B
-constexpr int kFine = 20;        // bins of the fine window (5 x 16 B)
 constexpr int kRound = kThreads * 32;   // tokens per select round (32 per thread)
 
 __host__ __device__ inline int dist_stride(int R) { return (R + 7) & ~7; }
@@ -71,34 +69,68 @@ struct DecodeArgs {
   int attend;
 };
 
+// Selection geometry of one kernel flavour.  Per-head selection (SH = false):
+// G selection heads, distances 0..384.  Shared selection (SH = true): one selection
+// per kv head over the sum of the G heads' distances, 0..384 G.
+template <int G, bool SH>
+struct Sel {
+  static constexpr int GS = SH ? 1 : G;                // selection heads
+  static constexpr int NB = SH ? 384 * G + 1 : kNBins;  // distance bins
+  static constexpr int BS = (NB + 3) / 4 * 4;           // histogram row stride (16 B multiple)
+  static constexpr int C = (NB + kNCoarse - 1) / kNCoarse;   // bins per coarse chunk
+  static constexpr int FW = (C + 4 + 3) / 4 * 4;        // fine-window bins (covers C + 1)
+  static constexpr int GM = SH ? (G < 4 ? G : 4) : 1;  // query heads (softmax states) per warp
+};
+
+// per-head selection: 385 bins, 30 coarse chunks of 13, a 20-bin (5 x 16 B) fine window
+static_assert(Sel<1, false>::NB == kNBins && Sel<1, false>::BS == kBinStride &&
+                  Sel<1, false>::C == 13 && Sel<1, false>::FW == 20,
+              "per-head selection geometry");
+static_assert(Sel<8, true>::NB <= 0x7fff, "summed distances must fit a signed 16-bit lane");
+
 struct SmemLayout {
   size_t ring, mbar, hist, coarse, fine, dist, list, qf, qc, qth, scan, merge, info, misc, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SmemLayout make_layout(int G, int R, int list_cap, int CS,
-                                                 int stages) {
+// GS, BS, FW, GM as in Sel<G, SH>; G = query heads of the unit.  With GM > 1 the
+// per-warp merge buffer (kWarps x GM partials) is placed in the ring region right
+// after the partials: the ring is idle once the scan is over, and rank 0 receives
+// the peers' partials only after the first cluster barrier.
+__host__ __device__ inline SmemLayout make_layout(int G, int GS, int BS, int FW, int GM, int R,
+                                                 int list_cap, int CS, int stages) {
   SmemLayout s;
   size_t o = 0;
   const size_t ring = size_t(stages) * kChunk * kCodeBytes;
-  const size_t part = size_t(CS) * G * kPartStride * 4;   // rank 0 receives the partials
+  const size_t merge = size_t(kWarps) * GM * kPartStride * 4;
+  const size_t part = size_t(CS) * G * kPartStride * 4 + (GM > 1 ? merge : 0);
   s.ring = o;  o = al(o + (ring > part ? ring : part), 128);
   s.mbar = o;  o = al(o + 8 * kMaxStages, 128);
-  s.hist = o;  o = al(o + size_t(G) * kBinStride * 4, 128);
-  s.coarse = o; o = al(o + size_t(CS) * G * kCoarseRow * 4, 128);   // pushed by the peers
-  s.fine = o;  o = al(o + size_t(CS) * G * kFine * 4, 128);         // pulled from the peers
-  s.dist = o;  o = al(o + size_t(G) * dist_stride(R) * 2, 128);
-  s.list = o;  o = al(o + size_t(G) * list_cap * 2, 128);
+  s.hist = o;  o = al(o + size_t(GS) * BS * 4, 128);
+  s.coarse = o; o = al(o + size_t(CS) * GS * kCoarseRow * 4, 128);   // pushed by the peers
+  s.fine = o;  o = al(o + size_t(CS) * GS * FW * 4, 128);            // pulled from the peers
+  s.dist = o;  o = al(o + size_t(GS) * dist_stride(R) * 2, 128);
+  s.list = o;  o = al(o + size_t(GS) * list_cap * 2, 128);
   s.qf = o;    o = al(o + size_t(G) * kD * 4, 128);
   s.qc = o;    o = al(o + size_t(G) * kCodeBytes, 128);
   s.qth = o;   o = al(o + size_t(G) * 12 * 4, 128);
-  s.scan = o;  o = al(o + size_t(2) * kWarps * G * 4, 128);
-  s.merge = o; o = al(o + size_t(kWarps) * kPartStride * 4, 128);
-  s.info = o;  o = al(o + size_t(G) * 9 * 4, 128);
+  s.scan = o;  o = al(o + size_t(2) * kWarps * GS * 4, 128);
+  if (GM > 1) {
+    s.merge = s.ring + size_t(CS) * G * kPartStride * 4;
+  } else {
+    s.merge = o; o = al(o + merge, 128);
+  }
+  s.info = o;  o = al(o + size_t(GS) * 9 * 4, 128);
   s.misc = o;  o = al(o + 128, 128);
   s.total = o;
   return s;
+}
+
+template <int G, bool SH>
+__host__ __device__ inline SmemLayout layout_of(int R, int list_cap, int CS, int stages) {
+  using X = Sel<G, SH>;
+  return make_layout(G, X::GS, X::BS, X::FW, X::GM, R, list_cap, CS, stages);
 }
 
 // Bit 15 and bit 31 of w0, then of w1, as bits 0..3 (the sign bits of four packed
@@ -151,28 +183,30 @@ __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t 
   }
 }
 
-template <int G, typename T>
+template <int G, bool SH, typename T>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a) {
+  using X = Sel<G, SH>;
+  constexpr int GS = X::GS, BS = X::BS, NB = X::NB, CB = X::C, FW = X::FW, GM = X::GM;
   extern __shared__ __align__(128) uint8_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = a.cluster;
   const int rank = int(cluster.block_rank());
   const int S = a.stages;
-  const SmemLayout lo = make_layout(G, a.keys_per_cta, a.list_cap, CS, S);
+  const SmemLayout lo = layout_of<G, SH>(a.keys_per_cta, a.list_cap, CS, S);
   uint8_t* ring = smem + lo.ring;
   float* part = reinterpret_cast<float*>(smem + lo.ring);           // [CS][G][kPartStride]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + lo.hist);    // [G][kBinStride]
-  uint32_t* coarse = reinterpret_cast<uint32_t*>(smem + lo.coarse);  // [CS][G][kCoarseRow]
-  uint32_t* fine = reinterpret_cast<uint32_t*>(smem + lo.fine);      // [CS][G][kFine]
-  uint16_t* dist = reinterpret_cast<uint16_t*>(smem + lo.dist);    // [G][RS]
-  uint16_t* list = reinterpret_cast<uint16_t*>(smem + lo.list);    // [G][list_cap]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + lo.hist);    // [GS][BS]
+  uint32_t* coarse = reinterpret_cast<uint32_t*>(smem + lo.coarse);  // [CS][GS][kCoarseRow]
+  uint32_t* fine = reinterpret_cast<uint32_t*>(smem + lo.fine);      // [CS][GS][FW]
+  uint16_t* dist = reinterpret_cast<uint16_t*>(smem + lo.dist);    // [GS][RS]
+  uint16_t* list = reinterpret_cast<uint16_t*>(smem + lo.list);    // [GS][list_cap]
   float* qf = reinterpret_cast<float*>(smem + lo.qf);              // [G][128]
   uint8_t* qc = smem + lo.qc;                                       // [G][32]
   uint32_t* qth = reinterpret_cast<uint32_t*>(smem + lo.qth);      // [G][12]
-  uint32_t* scan = reinterpret_cast<uint32_t*>(smem + lo.scan);    // [kWarps][G]
-  float* merge = reinterpret_cast<float*>(smem + lo.merge);        // [kWarps][kPartStride]
-  int* info = reinterpret_cast<int*>(smem + lo.info);              // [G][8]
+  uint32_t* scan = reinterpret_cast<uint32_t*>(smem + lo.scan);    // [2][kWarps][GS]
+  float* merge = reinterpret_cast<float*>(smem + lo.merge);        // [kWarps][GM][kPartStride]
+  int* info = reinterpret_cast<int*>(smem + lo.info);              // [GS][8], then [GS]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int unit = blockIdx.x / CS;
@@ -199,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   }
 
   // ---- prologue: zero histograms, encode (or fetch) the G query codes
-  for (int i = tid; i < G * kBinStride; i += kThreads) hist[i] = 0u;
+  for (int i = tid; i < GS * BS; i += kThreads) hist[i] = 0u;
   if (warp < G) {
     const int g = warp, h = kvh * G + g;
     if (a.qcodes != nullptr) {
@@ -257,6 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         Therm kt;
         make_therm(wd, kt);
+        uint32_t dsum = 0;   // shared selection: sum of the G heads' distances
 #pragma unroll
         for (int g0 = 0; g0 < G; g0 += GR) {
           if constexpr (G > 4) {
@@ -272,9 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 #pragma unroll
           for (int g = 0; g < GR; ++g) {
             const uint32_t dd = therm_dist_csa(kt, qreg[g], one);
-            dist[size_t(g0 + g) * RS + r] = static_cast<uint16_t>(dd);
-            atomicAdd(&hist[(g0 + g) * kBinStride + dd], 1u);
+            if constexpr (SH) {
+              dsum += dd;
+            } else {
+              dist[size_t(g0 + g) * RS + r] = static_cast<uint16_t>(dd);
+              atomicAdd(&hist[(g0 + g) * BS + dd], 1u);
+            }
           }
+        }
+        if constexpr (SH) {
+          dist[r] = static_cast<uint16_t>(dsum);
+          atomicAdd(&hist[dsum], 1u);
         }
       }
       // a slot is refilled only when the CTA's keys need more chunks than the ring
@@ -293,35 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   }
   __syncthreads();   // every key's distances and histogram counts are in
 
-  // ---- histograms -> inclusive cumulative histograms, in place (warp per head)
-  if (warp < G) {
-    uint32_t* row = hist + warp * kBinStride;
-    uint32_t loc[kCoarse];
-    uint32_t sum = 0;
-#pragma unroll
-    for (int i = 0; i < kCoarse; ++i) {
-      const int bin = kCoarse * lane + i;
-      loc[i] = bin < kNBins ? row[bin] : 0u;
-      sum += loc[i];
-    }
-    uint32_t inc = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    uint32_t run = inc - sum;
-#pragma unroll
-    for (int i = 0; i < kCoarse; ++i) {
-      const int bin = kCoarse * lane + i;
-      run += loc[i];
-      if (bin < kNBins) row[bin] = run;
-    }
-    // push this CTA's cumulative counts at the 30 coarse-chunk ends (+2 pad) into
-    // every peer, so the coarse level of the D* search reads local memory after
-    // the barrier.  Lane j now holds the count at the end of chunk j (lanes 29..31:
-    // the total); four lanes are gathered per 16-byte remote store.
-    const int g = warp;
+  // ---- histograms -> inclusive cumulative histograms, in place.  Then every CTA
+  // pushes its cumulative counts at the 30 coarse-chunk ends (+2 pad) into every
+  // peer, so the coarse level of the D* search reads local memory after the
+  // barrier: lane j of the pushing warp holds the count at the end of chunk j
+  // (lanes 30, 31: the total); four lanes are gathered per 16-byte remote store.
+  const auto push_coarse = [&](int g, uint32_t run) {
     const uint32_t c0 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 0);
     const uint32_t c1 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 1);
     const uint32_t c2 = __shfl_sync(0xffffffffu, run, (lane & 7) * 4 + 2);
@@ -329,62 +349,140 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     if (lane < kCoarseRow / 4) {
       for (int cc = 0; cc < CS; ++cc) {
         uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(coarse, cc) +
-                                              (size_t(rank) * G + g) * kCoarseRow) + lane;
+                                              (size_t(rank) * GS + g) * kCoarseRow) + lane;
         *dst = make_uint4(c0, c1, c2, c3);
       }
     }
+  };
+  if constexpr (CB <= 16) {
+    // 385 bins (per head, or one shared head of G = 1): a warp per selection head,
+    // lane l owning bins CB*l .. CB*l + CB-1 in registers
+    if (warp < GS) {
+      uint32_t* row = hist + warp * BS;
+      uint32_t loc[CB];
+      uint32_t sum = 0;
+#pragma unroll
+      for (int i = 0; i < CB; ++i) {
+        const int bin = CB * lane + i;
+        loc[i] = bin < NB ? row[bin] : 0u;
+        sum += loc[i];
+      }
+      uint32_t inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      uint32_t run = inc - sum;
+#pragma unroll
+      for (int i = 0; i < CB; ++i) {
+        const int bin = CB * lane + i;
+        run += loc[i];
+        if (bin < NB) row[bin] = run;
+      }
+      push_coarse(warp, run);
+    }
+  } else {
+    // wide shared-selection histogram (384 G + 1 bins, one row): the whole block,
+    // each thread owning PB consecutive bins read and written as 16-byte words
+    // (bins NB .. BS-1 are zero padding), one block scan
+    constexpr int PB = (NB + 4 * kThreads - 1) / (4 * kThreads) * 4;
+    uint32_t loc[PB];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int i4 = 0; i4 < PB; i4 += 4) {
+      const int bin = tid * PB + i4;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (bin < BS) v = *reinterpret_cast<const uint4*>(hist + bin);
+      loc[i4] = v.x; loc[i4 + 1] = v.y; loc[i4 + 2] = v.z; loc[i4 + 3] = v.w;
+      sum += v.x + v.y + v.z + v.w;
+    }
+    uint32_t ex[1] = {sum}, tot[1];
+    block_exclusive_scan<1>(ex, tot, scan, 0, lane, warp);
+    uint32_t run = ex[0];
+#pragma unroll
+    for (int i4 = 0; i4 < PB; i4 += 4) {
+      const int bin = tid * PB + i4;
+      uint4 v;
+      v.x = run += loc[i4];
+      v.y = run += loc[i4 + 1];
+      v.z = run += loc[i4 + 2];
+      v.w = run += loc[i4 + 3];
+      if (bin < BS) *reinterpret_cast<uint4*>(hist + bin) = v;
+    }
+    __syncthreads();
+    if (warp == 0) push_coarse(0, hist[min(CB * lane + CB - 1, NB - 1)]);
   }
 
   cluster.sync();   // cumulative histograms complete; coarse counts delivered
 
   // ---- resolve D*, the count selected in lower-ranked CTAs, and the ties taken.
   // Level 1 (local): the coarse chunk j* where the unit's cumulative count reaches
-  // k_eff.  Level 2: each peer's 20-bin window around chunk j* is pulled with
-  // 16-byte loads, then bins 13 j* - 1 .. 13 j* + 12 give D* exactly.
-  int* jst = info + G * 8;   // [G] coarse chunk per head
-  if (warp < G) {
+  // k_eff.  Level 2: each peer's FW-bin window around chunk j* is pulled with
+  // 16-byte loads, then bins CB j* - 1 .. CB j* + CB - 1 give D* exactly.
+  int* jst = info + GS * 8;   // [GS] coarse chunk per selection head
+  if (warp < GS) {
     const int g = warp;
     uint32_t S1 = 0;
     if (lane < kNCoarse) {
-      for (int cc = 0; cc < CS; ++cc) S1 += coarse[(cc * G + g) * kCoarseRow + lane];
+      for (int cc = 0; cc < CS; ++cc) S1 += coarse[(cc * GS + g) * kCoarseRow + lane];
     }
     const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < kNCoarse && S1 >= uint32_t(a.k_eff));
-    if (lane == 0) jst[g] = __ffs(hit1) - 1;   // exists: chunk 29 ends at bin 384, count L
+    if (lane == 0) jst[g] = __ffs(hit1) - 1;   // exists: chunk 29 ends at the last bin, count L
   }
   __syncthreads();
-  for (int i = tid; i < CS * G * (kFine / 4); i += kThreads) {
-    const int cc = i / (G * (kFine / 4));
-    const int g = (i / (kFine / 4)) % G;
-    const int q4 = i % (kFine / 4);
-    const int lo_bin = min(max(0, kCoarse * jst[g] - 1) & ~3, kBinStride - kFine);
+  for (int i = tid; i < CS * GS * (FW / 4); i += kThreads) {
+    const int cc = i / (GS * (FW / 4));
+    const int g = (i / (FW / 4)) % GS;
+    const int q4 = i % (FW / 4);
+    const int lo_bin = min(max(0, CB * jst[g] - 1) & ~3, BS - FW);
     const uint4 v = *(reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, cc) +
-                                                      g * kBinStride + lo_bin) + q4);
-    *(reinterpret_cast<uint4*>(fine + (cc * G + g) * kFine) + q4) = v;
+                                                      g * BS + lo_bin) + q4);
+    *(reinterpret_cast<uint4*>(fine + (cc * GS + g) * FW) + q4) = v;
   }
   __syncthreads();
-  if (warp < G) {
+  if (warp < GS) {
     const int g = warp;
     const uint32_t ke = uint32_t(a.k_eff);
     const int jstar = jst[g];
-    const int lo_bin = min(max(0, kCoarse * jstar - 1) & ~3, kBinStride - kFine);
-    // level 2: lane l -> bin 13 j* - 1 + l
-    const int d = kCoarse * jstar - 1 + lane;
-    uint32_t S2 = 0, Sb = 0;
-    if (lane < kCoarse + 1 && d >= 0) {
-      const int off = min(d, kNBins - 1) - lo_bin;
-      for (int cc = 0; cc < CS; ++cc) {
-        const uint32_t x = fine[(cc * G + g) * kFine + off];
-        S2 += x;
-        if (cc < rank) Sb += x;
+    const int lo_bin = min(max(0, CB * jstar - 1) & ~3, BS - FW);
+    // level 2, 32 bins per pass: lane l of pass p -> bin CB j* - 1 + 32 p + l.  The
+    // first bin reaching k_eff is D*; the counts one bin lower are the "less than"
+    // counts (carried across passes in lane 31's values).
+    int dstar = -1;
+    uint32_t less = 0, lt_before = 0, eq_before = 0, carry2 = 0, carryb = 0;
+    for (int base = 0; base < CB + 1 && dstar < 0; base += 32) {
+      const int l = base + lane;
+      const int d = CB * jstar - 1 + l;
+      uint32_t S2 = 0, Sb = 0;
+      if (l < CB + 1 && d >= 0) {
+        const int off = min(d, NB - 1) - lo_bin;
+        for (int cc = 0; cc < CS; ++cc) {
+          const uint32_t x = fine[(cc * GS + g) * FW + off];
+          S2 += x;
+          if (cc < rank) Sb += x;
+        }
       }
+      const uint32_t hit2 = __ballot_sync(0xffffffffu, l >= 1 && l < CB + 1 && S2 >= ke);
+      uint32_t p2 = __shfl_up_sync(0xffffffffu, S2, 1);
+      uint32_t pb = __shfl_up_sync(0xffffffffu, Sb, 1);
+      if (lane == 0) { p2 = carry2; pb = carryb; }
+      if (hit2) {
+        const int ls = __ffs(hit2) - 1;
+        dstar = CB * jstar - 1 + l - lane + ls;
+        less = __shfl_sync(0xffffffffu, p2, ls);        // unit count d < D*
+        lt_before = __shfl_sync(0xffffffffu, pb, ls);
+        eq_before = __shfl_sync(0xffffffffu, Sb, ls) - lt_before;
+      }
+      carry2 = __shfl_sync(0xffffffffu, S2, 31);
+      carryb = __shfl_sync(0xffffffffu, Sb, 31);
     }
-    const uint32_t hit2 = __ballot_sync(0xffffffffu, lane >= 1 && lane < kCoarse + 1 && S2 >= ke);
-    const int ls = __ffs(hit2) - 1;
-    const int dstar = kCoarse * jstar - 1 + ls;
-    const uint32_t less = __shfl_sync(0xffffffffu, S2, ls - 1);       // unit count d < D*
-    const uint32_t lt_before = __shfl_sync(0xffffffffu, Sb, ls - 1);
-    const uint32_t eq_before = __shfl_sync(0xffffffffu, Sb, ls) - lt_before;
-    const uint32_t* own = hist + g * kBinStride;
+    if (dstar < 0) {   // impossible when the counts are consistent; never index with it
+      if (lane == 0) atomicOr(a.err, kErrSelect);
+      dstar = NB - 1;
+      less = lt_before = eq_before = 0;
+    }
+    const uint32_t* own = hist + g * BS;
     const uint32_t lt_own = dstar > 0 ? own[dstar - 1] : 0u;
     const uint32_t eq_own = own[dstar] - lt_own;
     const uint32_t need = ke - less;                 // ties at D* the unit takes
@@ -404,43 +502,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   // tokens; one pass over the distances builds "< D*" and "== D*" bit masks, one
   // block scan ranks them, and only the selected bits are then visited
   {
-    int dstar[G], take[G], base[G], nsel[G];
+    int dstar[GS], take[GS], base[GS], nsel[GS];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < GS; ++g) {
       const int* in = info + g * 8;
       dstar[g] = in[0];
       base[g] = in[1];
       take[g] = in[2];
       nsel[g] = in[3];
     }
-    uint32_t carry_lt[G], carry_eq[G];
+    uint32_t carry_lt[GS], carry_eq[GS];
 #pragma unroll
-    for (int g = 0; g < G; ++g) carry_lt[g] = carry_eq[g] = 0;
+    for (int g = 0; g < GS; ++g) carry_lt[g] = carry_eq[g] = 0;
     for (int rb = 0, parity = 0; rb < n; rb += kRound, parity ^= 1) {
       const int nr = min(kRound, n - rb);
       const int per = (((nr + kThreads - 1) / kThreads) + 7) & ~7;   // multiple of 8, <= 32
       const int s0 = rb + tid * per;
       const int cntv = max(0, min(per, rb + nr - s0));
-      uint32_t ltm[G], eqm[G], cnt[G], tot[G];
+      uint32_t ltm[GS], eqm[GS], cnt[GS], tot[GS];
       const uint32_t valid = cntv >= 32 ? 0xffffffffu : ((1u << cntv) - 1u);
       // packed compares, two distances per word: in each 16-bit lane
       // (0x8000 + D*) - d keeps bit 15 iff d <= D*, (0x7fff + D*) - d iff d < D*
-      // (distances <= 384, so no lane borrows from its neighbour).  All G heads'
-      // loads of a group of 8 positions are issued before any compare.
-      uint32_t cle[G], clt[G];
+      // (distances <= 384 G <= 3072, so no lane borrows from its neighbour).  All
+      // selection heads' loads of a group of 8 positions are issued before any compare.
+      uint32_t cle[GS], clt[GS];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int g = 0; g < GS; ++g) {
         cle[g] = (0x8000u + uint32_t(dstar[g])) * 0x10001u;
         clt[g] = cle[g] - 0x10001u;
         ltm[g] = eqm[g] = 0;
       }
       for (int i8 = 0; i8 < cntv; i8 += 8) {
-        uint4 v[G];
+        uint4 v[GS];
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int g = 0; g < GS; ++g)
           v[g] = *reinterpret_cast<const uint4*>(dist + size_t(g) * RS + s0 + i8);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
+        for (int g = 0; g < GS; ++g) {
           const uint32_t l0 = lane_sign_bits(clt[g] - v[g].x, clt[g] - v[g].y);
           const uint32_t l1 = lane_sign_bits(clt[g] - v[g].z, clt[g] - v[g].w);
           const uint32_t e0 = lane_sign_bits(cle[g] - v[g].x, cle[g] - v[g].y) & ~l0;
@@ -450,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         }
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int g = 0; g < GS; ++g) {
         ltm[g] &= valid;
         eqm[g] &= valid;
         cnt[g] = (uint32_t(__popc(ltm[g])) << 16) | uint32_t(__popc(eqm[g]));
@@ -467,9 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           }
         }
       }
-      block_exclusive_scan<G>(cnt, tot, scan, parity, lane, warp);
+      block_exclusive_scan<GS>(cnt, tot, scan, parity, lane, warp);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int g = 0; g < GS; ++g) {
         const int lt_b = int(carry_lt[g] + (cnt[g] >> 16));
         const int eq_b = int(carry_eq[g] + (cnt[g] & 0xffffu));
         // this thread's ties that still fit: the lowest (take - eq_b) bits of eqm
@@ -482,9 +580,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         }
         uint32_t sel = ltm[g] | sel_eq;
         int rk = lt_b + min(eq_b, take[g]);
-        int32_t* orow = a.idx_out != nullptr
-                            ? a.idx_out + (int64_t(b) * a.Hq + kvh * G + g) * a.k_eff + base[g]
-                            : nullptr;
+        // idx_out rows: [B][Hq] for per-head selection, [B][Hkv] for shared selection
+        const int64_t orow_id = SH ? int64_t(b) * a.Hkv + kvh : int64_t(b) * a.Hq + kvh * G + g;
+        int32_t* orow = a.idx_out != nullptr ? a.idx_out + orow_id * a.k_eff + base[g] : nullptr;
         uint16_t* lrow = list + size_t(g) * a.list_cap;
         while (sel) {
           const int i = __ffs(sel) - 1;
@@ -505,30 +603,52 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   }
   __syncthreads();
 
-  // ---- attention over the selected rows: this CTA's split of the unit's softmax
+  // ---- attention over the selected rows: this CTA's split of the unit's softmax.
+  // The warps form G / GM groups; group gi serves query heads gi GM .. gi GM + GM-1,
+  // its warps taking rows sub, sub + WPG, ... of the heads' list.  Per-head
+  // selection: GM = 1, one group per head.  Shared selection: one list, GM <= 4
+  // heads scored per loaded K/V row (for G = 8 the second group's reads of a row
+  // hit L2).
   if (a.attend) {
-    constexpr int WPH = kWarps / G;   // warps per head
-    const int g = warp % G, sub = warp / G;
-    const int nsel = info[g * 8 + 3];
-    const uint16_t* lrow = list + size_t(g) * a.list_cap;
-    const float* qrow = qf + g * kD + 4 * lane;
-    const float qv[4] = {qrow[0], qrow[1], qrow[2], qrow[3]};
+    constexpr int NGR = G / GM;          // warp groups
+    constexpr int WPG = kWarps / NGR;    // warps per group
+    const int gi = warp % NGR, sub = warp / NGR;
+    const int sel_head = SH ? 0 : gi;
+    const int nsel = info[sel_head * 8 + 3];
+    const uint16_t* lrow = list + size_t(sel_head) * a.list_cap;
     const T* kb = static_cast<const T*>(a.k) + int64_t(unit) * a.Lmax * kD;
     const T* vb = static_cast<const T*>(a.v) + int64_t(unit) * a.Lmax * kD;
-    SoftmaxState st;
-    st.init();
-    attend_rows<T>(kb, vb, nsel, sub, WPH, [&](int j) { return p0 + int64_t(lrow[j]); }, qv,
-                   a.scale_log2, lane, st);
-    float* mw = merge + warp * kPartStride;
-    if (lane == 0) { mw[0] = st.m; mw[1] = st.l; }
+    float qv[GM][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) mw[4 + 4 * lane + r] = st.acc[r];
+    for (int h = 0; h < GM; ++h) {
+      const float* qrow = qf + (gi * GM + h) * kD + 4 * lane;
+      qv[h][0] = qrow[0]; qv[h][1] = qrow[1]; qv[h][2] = qrow[2]; qv[h][3] = qrow[3];
+    }
+    SoftmaxState st[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) st[h].init();
+    const auto pos_of = [&](int j) { return p0 + int64_t(lrow[j]); };
+    if constexpr (GM == 1) {
+      attend_rows<T>(kb, vb, nsel, sub, WPG, pos_of, qv[0], a.scale_log2, lane, st[0]);
+    } else {
+      constexpr int kRowsG = GM <= 2 ? 8 : 4;
+      attend_rows_group<T, GM, kRowsG>(kb, vb, nsel, sub, WPG, pos_of, qv, a.scale_log2, lane,
+                                       st);
+    }
+    // merge row (sub * G + head) holds warp `sub` of the head's group's partial
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      float* mw = merge + (sub * G + gi * GM + h) * kPartStride;
+      if (lane == 0) { mw[0] = st[h].m; mw[1] = st[h].l; }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) mw[4 + 4 * lane + r] = st[h].acc[r];
+    }
     __syncthreads();
     float* dstp = cluster.map_shared_rank(part, 0) + size_t(rank) * G * kPartStride;
     for (int i = tid; i < G * kD; i += kThreads) {
       const int gg = i / kD, dim = i % kD;
       float M = -INFINITY, Ls = 0.f, A = 0.f;
-      for (int sw = 0; sw < WPH; ++sw) {
+      for (int sw = 0; sw < WPG; ++sw) {
         const float* mm = merge + (sw * G + gg) * kPartStride;
         merge_into(mm[0], mm[1], mm[4 + dim], M, Ls, A);
       }
@@ -567,25 +687,25 @@ static int max_smem_optin(int dev) {
   return v;
 }
 
-template <int G, typename T>
+template <int G, bool SH, typename T>
 static cudaError_t prepare_kernel() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     int dev = 0;
     cudaGetDevice(&dev);
-    err = cudaFuncSetAttribute(decode_kernel<G, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               max_smem_optin(dev));
+    err = cudaFuncSetAttribute(decode_kernel<G, SH, T>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem_optin(dev));
     if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(decode_kernel<G, T>,
+      err = cudaFuncSetAttribute(decode_kernel<G, SH, T>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   });
   return err;
 }
 
-template <int G, typename T>
+template <int G, bool SH, typename T>
 static int active_clusters_g(int cs, size_t smem) {
-  if (prepare_kernel<G, T>() != cudaSuccess) return 0;
+  if (prepare_kernel<G, SH, T>() != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs);
   cfg.blockDim = dim3(kThreads);
@@ -598,28 +718,49 @@ static int active_clusters_g(int cs, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int nclusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, T>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, SH, T>, &cfg) !=
+      cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
   return nclusters;
 }
 
-static int active_clusters(int G, int cs, size_t smem) {
+template <bool SH>
+static int active_clusters_s(int G, int cs, size_t smem) {
   switch (G) {
-    case 1: return active_clusters_g<1, __nv_bfloat16>(cs, smem);
-    case 2: return active_clusters_g<2, __nv_bfloat16>(cs, smem);
-    case 4: return active_clusters_g<4, __nv_bfloat16>(cs, smem);
-    case 8: return active_clusters_g<8, __nv_bfloat16>(cs, smem);
+    case 1: return active_clusters_g<1, SH, __nv_bfloat16>(cs, smem);
+    case 2: return active_clusters_g<2, SH, __nv_bfloat16>(cs, smem);
+    case 4: return active_clusters_g<4, SH, __nv_bfloat16>(cs, smem);
+    case 8: return active_clusters_g<8, SH, __nv_bfloat16>(cs, smem);
   }
   return 0;
+}
+
+static int active_clusters(int G, bool shared, int cs, size_t smem) {
+  return shared ? active_clusters_s<true>(G, cs, smem) : active_clusters_s<false>(G, cs, smem);
+}
+
+static size_t layout_total(int G, bool shared, int R, int list_cap, int cs, int stages) {
+#define ADAMAS_LAYOUT_CASE(GG)                                                        \
+  case GG:                                                                            \
+    return shared ? layout_of<GG, true>(R, list_cap, cs, stages).total                \
+                  : layout_of<GG, false>(R, list_cap, cs, stages).total;
+  switch (G) {
+    ADAMAS_LAYOUT_CASE(1)
+    ADAMAS_LAYOUT_CASE(2)
+    ADAMAS_LAYOUT_CASE(4)
+    ADAMAS_LAYOUT_CASE(8)
+  }
+#undef ADAMAS_LAYOUT_CASE
+  return ~size_t(0);
 }
 
 // Chooses the cluster size: among sizes whose shared memory fits (and, on a device,
 // whose clusters can be scheduled), the one with the least modelled time
 // waves x (per-key scan cost x keys per CTA + fixed per-wave latency).
-bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int smem_cap,
-                      bool query_device, Plan& p) {
+bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int sms,
+                      int smem_cap, bool query_device, Plan& p) {
   const int G = Hq / Hkv;
   const int64_t U = int64_t(B) * Hkv;
   const int64_t k_eff = std::min<int64_t>(k, L);
@@ -632,12 +773,12 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int sme
     const int list_cap = int(std::max<int64_t>(1, std::min<int64_t>(R, k_eff)));
     const int64_t nchunks = (R + kChunk - 1) / kChunk;
     int stages = int(std::min<int64_t>(kMaxStages, std::max<int64_t>(1, nchunks)));
-    while (stages > 1 && make_layout(G, int(R), list_cap, cs, stages).total > size_t(smem_cap))
+    while (stages > 1 && layout_total(G, shared, int(R), list_cap, cs, stages) > size_t(smem_cap))
       --stages;
-    const size_t smem = make_layout(G, int(R), list_cap, cs, stages).total;
+    const size_t smem = layout_total(G, shared, int(R), list_cap, cs, stages);
     if (smem > size_t(smem_cap)) continue;
     int conc_clusters = sms / cs;
-    if (query_device) conc_clusters = active_clusters(G, cs, smem);
+    if (query_device) conc_clusters = active_clusters(G, shared, cs, smem);
     if (conc_clusters < 1) continue;
     const int64_t total = U * cs;
     const int64_t conc = int64_t(conc_clusters) * cs;
@@ -659,23 +800,24 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int sme
   return found && p.grid > 0 && int64_t(p.grid) == U * p.cluster && U * p.cluster < (1ll << 31);
 }
 
-bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, Plan& p) {
+bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
+                                    Plan& p) {
   int dev = 0;
   const int sms = current_device_sms(&dev);
   if (sms <= 0) {
     // no device visible: plan for a 148-SM part with the sm_100 shared-memory cap
-    return make_decode_plan(B, Hq, Hkv, L, k, 148, 232448, false, p);
+    return make_decode_plan(B, Hq, Hkv, L, k, shared, 148, 232448, false, p);
   }
-  return make_decode_plan(B, Hq, Hkv, L, k, sms, max_smem_optin(dev), true, p);
+  return make_decode_plan(B, Hq, Hkv, L, k, shared, sms, max_smem_optin(dev), true, p);
 }
 
 // The decode workspace only carries the device error word (bounded copy waits).
 size_t decode_workspace_bytes(int, int, int, int64_t, int) { return 256; }
 size_t decode_workspace_error_offset() { return 8; }
 
-template <int G, typename T>
+template <int G, bool SH, typename T>
 static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t stream) {
-  const cudaError_t e = prepare_kernel<G, T>();
+  const cudaError_t e = prepare_kernel<G, SH, T>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
@@ -689,16 +831,16 @@ static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t str
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<G, T>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<G, SH, T>, a);
 }
 
-template <typename T>
+template <bool SH, typename T>
 static cudaError_t launch_t(int G, const DecodeArgs& a, const Plan& p, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_g<1, T>(a, p, s);
-    case 2: return launch_g<2, T>(a, p, s);
-    case 4: return launch_g<4, T>(a, p, s);
-    case 8: return launch_g<8, T>(a, p, s);
+    case 1: return launch_g<1, SH, T>(a, p, s);
+    case 2: return launch_g<2, SH, T>(a, p, s);
+    case 4: return launch_g<4, SH, T>(a, p, s);
+    case 8: return launch_g<8, SH, T>(a, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -706,7 +848,8 @@ static cudaError_t launch_t(int G, const DecodeArgs& a, const Plan& p, cudaStrea
 cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
                           int64_t Lmax, int64_t L, int kk, float t, void* ws,
-                          int32_t* idx_out, float* out, const Plan& p, cudaStream_t stream) {
+                          int32_t* idx_out, float* out, bool shared, const Plan& p,
+                          cudaStream_t stream) {
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q; a.qcodes = qcodes; a.k = k; a.v = v; a.codes = codes;
@@ -721,8 +864,12 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.list_cap = p.list_cap;
   a.stages = p.stages;
   a.attend = out != nullptr ? 1 : 0;
-  if (dt == ADAMAS_F32) return launch_t<float>(G, a, p, stream);
-  return launch_t<__nv_bfloat16>(G, a, p, stream);
+  if (shared) {
+    if (dt == ADAMAS_F32) return launch_t<true, float>(G, a, p, stream);
+    return launch_t<true, __nv_bfloat16>(G, a, p, stream);
+  }
+  if (dt == ADAMAS_F32) return launch_t<false, float>(G, a, p, stream);
+  return launch_t<false, __nv_bfloat16>(G, a, p, stream);
 }
 
 }  // namespace adamas

@@ -65,13 +65,15 @@ class Workload:
     def elem_bytes(self) -> int:
         return 4 if self.dtype == torch.float32 else 2
 
-    def algorithmic_bytes(self, k: int) -> int:
+    def algorithmic_bytes(self, k: int, shared: bool = False) -> int:
         """Bytes one decode step must move per layer: codes scanned, selected K+V
-        rows per query head, q read and fp32 output written."""
+        rows per query head (per kv head when the selection is shared by the
+        group), q read and fp32 output written."""
         k_eff = min(k, self.L)
         e = self.elem_bytes
+        sel_rows = self.B * (self.Hkv if shared else self.Hq) * k_eff
         return (self.B * self.Hkv * self.L * (self.d // 4)
-                + self.B * self.Hq * k_eff * 2 * self.d * e
+                + sel_rows * 2 * self.d * e
                 + self.B * self.Hq * self.d * e
                 + self.B * self.Hq * self.d * 4)
 

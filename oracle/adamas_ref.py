@@ -247,3 +247,41 @@ def decode_step_shared(q: np.ndarray, K: np.ndarray, V: np.ndarray, k: int, t: f
                 h = kvh * G + g
                 out[b, h] = sparse_attention(q[b, h], K[b, kvh, :L], V[b, kvh, :L], sel)
     return idx, out
+
+
+# ------------------------------------- per-sequence context lengths (serving form)
+def decode_step_varlen(q: np.ndarray, K: np.ndarray, V: np.ndarray, seq_lens, k: int,
+                       t: float, key_codes: np.ndarray | None = None,
+                       query_codes: np.ndarray | None = None, shared: bool = False):
+    """Decode step where sequence b has its own context length seq_lens[b].
+
+    The pages run every sequence over its own context; nothing in the method
+    changes: sequence b is decode_step (or decode_step_shared) over its first
+    seq_lens[b] positions.  The result is laid out for a batch:
+    idx [B, rows, min(k, Lmax)] with entries past min(k, seq_lens[b]) set to -1
+    (rows = Hq, or Hkv when shared), out [B, Hq, d]; a sequence of length 0 selects
+    nothing and its output is all zeros (a reading: softmax over an empty set is
+    undefined).  K, V: [B, Hkv, Lmax, d] logical caches; paging is only a storage
+    layout and is not modelled here.
+    """
+    q = np.asarray(q)
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = K.shape
+    seq_lens = [int(x) for x in seq_lens]
+    if len(seq_lens) != B or min(seq_lens) < 0 or max(seq_lens) > Lmax:
+        raise ValueError("seq_lens must hold B lengths in [0, Lmax]")
+    k_row = min(int(k), Lmax)
+    rows = Hkv if shared else Hq
+    idx = np.full((B, rows, k_row), -1, dtype=np.int64)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    step = decode_step_shared if shared else decode_step
+    for b, Lb in enumerate(seq_lens):
+        if Lb == 0:
+            continue
+        kc = None if key_codes is None else np.asarray(key_codes)[b:b + 1, :, :Lb]
+        qc = None if query_codes is None else np.asarray(query_codes)[b:b + 1]
+        ib, ob = step(q[b:b + 1], K[b:b + 1, :, :Lb], V[b:b + 1, :, :Lb], k, t,
+                      key_codes=kc, query_codes=qc)
+        idx[b, :, :ib.shape[-1]] = ib[0]
+        out[b] = ob[0]
+    return idx, out

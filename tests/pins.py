@@ -17,6 +17,9 @@ What pins what:
 * Attention: budget = L equals torch's dense scaled-dot-product attention; budget 1
   returns the V row.
 * GQA mapping and recall of planted keys on the seeded single-head workload.
+* Shared selection: G = 1 reduction, pure-Python brute force, identical heads.
+* Per-sequence lengths: pure-Python brute force (empty, short and long sequences,
+  -1 padding), invariance to cache slots past a length, full-length reduction.
 """
 from __future__ import annotations
 
@@ -301,6 +304,89 @@ def check_shared_identical_heads():
     assert np.allclose(o_sh, o_head, atol=1e-12)
 
 
+# ------------------------------------------- per-sequence context lengths
+def _brute_select(dist, k):
+    return sorted(sorted(range(len(dist)), key=lambda j: (dist[j], j))[:k])
+
+
+def _dense(qv, Ks, Vs):
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(qv)[None, None, None, :], torch.from_numpy(Ks)[None, None],
+        torch.from_numpy(Vs)[None, None])[0, 0, 0].numpy()
+
+
+def check_varlen_bruteforce():
+    """Lengths 0, 5, 37 in a 40-slot cache: per head, a pure-Python Manhattan
+    distance over the sequence's own positions, full sort by (distance, position),
+    dense attention over the selection; -1 padding past min(k, L_b); an empty
+    sequence selects nothing and outputs zeros.  Same for the shared selection with
+    the group's distances summed."""
+    rng = np.random.default_rng(43)
+    B, Hq, Hkv, Lmax, k, t = 3, 4, 2, 40, 8, 0.35
+    G = Hq // Hkv
+    lens = [0, 5, 37]
+    q = rng.standard_normal((B, Hq, 128))
+    K = rng.standard_normal((B, Hkv, Lmax, 128))
+    V = rng.standard_normal((B, Hkv, Lmax, 128))
+    cq = ref.unpack_codes(ref.encode(q, t))
+    ck = ref.unpack_codes(ref.encode(K, t))
+
+    def dist(b, h, kvh, Lb):
+        return [sum(abs(int(cq[b, h, i]) - int(ck[b, kvh, j, i])) for i in range(128))
+                for j in range(Lb)]
+
+    idx, out = ref.decode_step_varlen(q, K, V, lens, k, t)
+    sidx, sout = ref.decode_step_varlen(q, K, V, lens, k, t, shared=True)
+    assert idx.shape == (B, Hq, k) and sidx.shape == (B, Hkv, k)
+    for b, Lb in enumerate(lens):
+        ke = min(k, Lb)
+        for kvh in range(Hkv):
+            per = [dist(b, kvh * G + g, kvh, Lb) for g in range(G)]
+            swant = _brute_select([sum(c) for c in zip(*per)], k) if Lb else []
+            assert list(sidx[b, kvh, :ke]) == swant and (sidx[b, kvh, ke:] == -1).all()
+            for g in range(G):
+                h = kvh * G + g
+                want = _brute_select(per[g], k) if Lb else []
+                assert list(idx[b, h, :ke]) == want, (b, h)
+                assert (idx[b, h, ke:] == -1).all()
+                if Lb == 0:
+                    assert (out[b, h] == 0).all() and (sout[b, h] == 0).all()
+                    continue
+                assert np.allclose(out[b, h], _dense(q[b, h], K[b, kvh, want], V[b, kvh, want]),
+                                   atol=1e-12)
+                assert np.allclose(sout[b, h],
+                                   _dense(q[b, h], K[b, kvh, swant], V[b, kvh, swant]),
+                                   atol=1e-12)
+
+
+def check_varlen_ignores_tail():
+    """Cache slots at or past a sequence's length take no part: overwriting them
+    changes neither the selection nor the output."""
+    rng = np.random.default_rng(47)
+    B, Hq, Hkv, Lmax = 2, 2, 1, 64
+    lens = [30, 64]
+    q = rng.standard_normal((B, Hq, 128))
+    K = rng.standard_normal((B, Hkv, Lmax, 128))
+    V = rng.standard_normal((B, Hkv, Lmax, 128))
+    i1, o1 = ref.decode_step_varlen(q, K, V, lens, 12, 0.5)
+    K2, V2 = K.copy(), V.copy()
+    K2[0, :, 30:] = np.repeat(q[0, :1, None, :], 34, axis=1) * 3.0   # would win if scanned
+    V2[0, :, 30:] = 1e6
+    i2, o2 = ref.decode_step_varlen(q, K2, V2, lens, 12, 0.5)
+    assert np.array_equal(i1, i2) and np.array_equal(o1, o2)
+
+
+def check_varlen_uniform_is_decode_step():
+    """Every sequence at full length: the batch step of decode_step."""
+    rng = np.random.default_rng(53)
+    q = rng.standard_normal((2, 4, 128))
+    K = rng.standard_normal((2, 2, 50, 128))
+    V = rng.standard_normal((2, 2, 50, 128))
+    i1, o1 = ref.decode_step(q, K, V, 16, 0.5)
+    i2, o2 = ref.decode_step_varlen(q, K, V, [50, 50], 16, 0.5)
+    assert np.array_equal(i1, i2) and np.array_equal(o1, o2)
+
+
 ALL_CHECKS = [
     check_hadamard_matches_scipy, check_hadamard_orthogonal,
     check_rotate_involution_and_dot, check_rotate_closed_forms, check_bucket_golden,
@@ -309,4 +395,5 @@ ALL_CHECKS = [
     check_attention_dense, check_attention_budget1, check_decode_dense_limit,
     check_gqa_and_planted, check_planted_recall_single_head,
     check_shared_g1_is_per_head, check_shared_bruteforce, check_shared_identical_heads,
+    check_varlen_bruteforce, check_varlen_ignores_tail, check_varlen_uniform_is_decode_step,
 ]

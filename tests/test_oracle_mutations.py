@@ -11,7 +11,8 @@ from pins import ALL_CHECKS
 
 _orig = {name: getattr(ref, name) for name in (
     "sylvester_hadamard", "hadamard_rotate", "bucketize", "pack_codes", "unpack_codes",
-    "manhattan", "select_topk", "sparse_attention", "decode_step", "decode_step_shared")}
+    "manhattan", "select_topk", "sparse_attention", "decode_step", "decode_step_shared",
+    "decode_step_varlen")}
 
 
 def _h_or(n=128):                      # popcount(i | j) instead of i & j
@@ -114,6 +115,26 @@ def _shared_first_head_only(q, K, V, k, t, key_codes=None, query_codes=None):
     return idx, out
 
 
+def _varlen_full_cache(q, K, V, seq_lens, k, t, key_codes=None, query_codes=None,
+                      shared=False):
+    # every non-empty sequence scanned over the whole cache instead of its length
+    lens = [K.shape[2] if int(x) else 0 for x in seq_lens]
+    return _orig["decode_step_varlen"](q, K, V, lens, k, t, shared=shared)
+
+
+def _varlen_zero_pad(q, K, V, seq_lens, k, t, key_codes=None, query_codes=None, shared=False):
+    # unused index slots padded with 0 instead of -1
+    idx, out = _orig["decode_step_varlen"](q, K, V, seq_lens, k, t, shared=shared)
+    return np.where(idx < 0, 0, idx), out
+
+
+def _varlen_off_by_one(q, K, V, seq_lens, k, t, key_codes=None, query_codes=None,
+                       shared=False):
+    # one slot past the length scanned as well
+    lens = [min(int(x) + 1, K.shape[2]) if int(x) else 0 for x in seq_lens]
+    return _orig["decode_step_varlen"](q, K, V, lens, k, t, shared=shared)
+
+
 MUTATIONS = {
     "hadamard_or": ("sylvester_hadamard", _h_or),
     "rotate_unscaled": ("hadamard_rotate", _rotate_unscaled),
@@ -129,6 +150,9 @@ MUTATIONS = {
     "attention_k_as_v": ("sparse_attention", _attn_uses_k),
     "decode_gqa_modulo": ("decode_step", _decode_mod_gqa),
     "shared_first_head_only": ("decode_step_shared", _shared_first_head_only),
+    "varlen_full_cache": ("decode_step_varlen", _varlen_full_cache),
+    "varlen_zero_pad": ("decode_step_varlen", _varlen_zero_pad),
+    "varlen_off_by_one": ("decode_step_varlen", _varlen_off_by_one),
 }
 
 

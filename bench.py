@@ -1,7 +1,7 @@
 """Benchmark of the Adamas decode step on B200: µs per step and effective HBM GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--budget 128]
-                    [--shared] [--impl ours|reference]
+                    [--shared] [--paged PAGE] [--impl ours|reference]
 
 Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32 query / 8 kv heads,
 d = 128, context 32768, bf16 K/V with 4 outlier channels, budget 128.  A "step" is
@@ -182,6 +182,24 @@ def run_ours(args, rank, world, local):
     step_bytes = w.algorithmic_bytes(k, shared) * w.layers
     if append:
         step_bytes += w.B * w.Hkv * append * (128 * w.elem_bytes + 32)
+    pc = None
+    if args.paged:
+        # the same caches held in a page pool (shuffled pages, block table, lengths);
+        # an append re-encodes the pages that hold the new positions
+        from workloads.paging import make_block_table, scatter_to_pages
+        ps = args.paged
+        pc = make_block_table([L] * w.B, L, ps, seed=args.config, spare=0)
+        bt = pc.block_table.to(dev)
+        lens = pc.seq_lens.to(dev)
+        app_ids = (pc.block_table[:, (L - append) // ps:(L + ps - 1) // ps].reshape(-1)
+                   .contiguous().to(dev) if append else None)
+        paged_sets = []
+        while layer_sets:
+            q, kc, vc, cd = layer_sets.pop(0)
+            paged_sets.append((q, scatter_to_pages(kc, pc), scatter_to_pages(vc, pc),
+                               scatter_to_pages(cd, pc)))
+            del kc, vc, cd
+        layer_sets = paged_sets
     R = args.replicas or replicas_for_l2(step_bytes, l2, 2.0)
     sets = [layer_sets]
     for _ in range(R - 1):
@@ -192,12 +210,19 @@ def run_ours(args, rank, world, local):
     plan = (ad.decode_plan_shared if shared else ad.decode_plan)(w.B, w.Hq, w.Hkv, L, k)
     launches_per_step = w.layers * (2 if append else 1)
 
-    def step(i, s, q_override=None):
+    def step(i, s, q_override=None, out_t=None):
         for (q, kc, vc, cd) in sets[i % R]:
+            qq = q if q_override is None else q_override
+            o = out if out_t is None else out_t
+            if pc is not None:
+                if append:
+                    ad.encode_pages(kc, cd, t, page_ids=app_ids, stream=s)
+                ad.decode_step_paged(qq, kc, vc, cd, bt, lens, L, k, t, ws, shared=shared, out=o,
+                                     stream=s)
+                continue
             if append:
                 ad.encode_keys(kc, cd, L - append, append, t, stream=s)
-            decode(q if q_override is None else q_override, kc, vc, cd, L, k, t, ws, out=out,
-                   stream=s)
+            decode(qq, kc, vc, cd, L, k, t, ws, out=o, stream=s)
 
     # eager warm-up (also loads the kernels and sets their attributes)
     with torch.cuda.stream(stream):
@@ -275,11 +300,23 @@ def run_ours(args, rank, world, local):
 
     # per layer one C call: pinned q in, fused decode, fp32 out back to pinned host;
     # the calls are bound to their buffers once, as a serving loop would
-    calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws, outs[li],
-                                    out_host[li], stream=stream, shared=shared)
-              for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
+    calls = None
+    if pc is None:
+        calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws,
+                                        outs[li], out_host[li], stream=stream, shared=shared)
+                  for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
 
     def e2e_step(i):
+        if calls is None:
+            # paged caches: the host copies around the public paged entry point
+            q_dev.copy_(q_host, non_blocking=True)
+            for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
+                if append:
+                    ad.encode_pages(kc, cd, t, page_ids=app_ids, stream=stream)
+                ad.decode_step_paged(q_dev[li], kc, vc, cd, bt, lens, L, k, t, ws, shared=shared,
+                                     out=outs[li], stream=stream)
+            out_host.copy_(outs, non_blocking=True)
+            return
         for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
             if append:
                 ad.encode_keys(kc, cd, L - append, append, t, stream=stream)
@@ -404,6 +441,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shared", action="store_true",
                     help="shared GQA selection (one top-k per kv head)")
+    ap.add_argument("--paged", type=int, default=0, metavar="PAGE",
+                    help="hold the caches in a pool of PAGE-token pages (block tables)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.budget is None:
@@ -426,7 +465,8 @@ def main():
     gbs_rank = aggregate_gbs(r["step_bytes"], per_step_s, 1)
     value = aggregate_gbs(r["step_bytes"], per_step_s, world)
     e2e_step_s = r["ms_e2e"] / 1e3 / r["K2"]
-    key = f"config{args.config}_k{k}" + ("_shared" if args.shared else "")
+    key = (f"config{args.config}_k{k}" + ("_shared" if args.shared else "")
+           + (f"_paged{args.paged}" if args.paged else ""))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -445,6 +485,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128, "L": w.L,
                    "k": k, "algorithmic_bytes_per_step": r["step_bytes"],
                    "selection": "shared per kv head" if args.shared else "per query head",
+                   "cache": f"paged, {args.paged}-token pages" if args.paged else "contiguous",
                    "replicas": r["R"], "l2": "rotated replicas, working set >= 2x L2",
                    "layers": w.layers, "append_tokens": w.append,
                    "graph": r["use_graph"], "ctas": r["plan"]["ctas"],

@@ -102,7 +102,9 @@ adamas_status adamas_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stre
  * SYNCHRONIZES `stream`, then reads the device error word of a decode workspace.
  * Returns ADAMAS_ERR_TIMEOUT if a kernel gave up a bounded wait (completion of a
  * bulk copy into shared memory) since the workspace was initialised,
- * ADAMAS_ERR_INTERNAL if the top-k bookkeeping of a kernel found no k-th distance
+ * ADAMAS_ERR_INVALID_ARG if a kernel met a device-resident length or page id out of
+ * range (adamas_decode_step_varlen / _paged), ADAMAS_ERR_INTERNAL if the top-k
+ * bookkeeping of a kernel found no k-th distance
  * (inconsistent counts: a bug, never expected), else ADAMAS_OK (or ADAMAS_ERR_CUDA
  * if the stream reported an error).
  */
@@ -182,6 +184,68 @@ adamas_status adamas_select_topk_shared(const uint8_t* qcodes, const uint8_t* co
                                         int Hq, int Hkv, int64_t Lmax, int64_t L, int k,
                                         void* workspace, size_t ws_bytes, int32_t* idx_out,
                                         cudaStream_t stream);
+
+/*
+ * Per-sequence context lengths (serving form of the same step; the Adamas pages run
+ * each sequence over its own context and the method is unchanged).  Contiguous
+ * caches as in adamas_decode_step, [B][Hkv][Lmax][d]; sequence b uses its first
+ * seq_lens[b] positions (device array [B] of int32, each in [0, Lmax]).  shared = 0
+ * selects per query head (idx_out [B][Hq][min(k, Lmax)]), shared = 1 per kv head
+ * as adamas_decode_step_shared (idx_out [B][Hkv][min(k, Lmax)]).  A row holds the
+ * min(k, seq_lens[b]) selected positions, ascending, then -1.  A sequence of length
+ * 0 selects nothing and its output is all zeros.  The launch plan is made for Lmax.
+ * A length outside [0, Lmax] is read on the device: it is clamped and recorded in
+ * the workspace error word (adamas_check_workspace returns ADAMAS_ERR_INVALID_ARG).
+ */
+adamas_status adamas_decode_step_varlen(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, const int32_t* seq_lens,
+                                        int k, float t, int shared, void* workspace,
+                                        size_t ws_bytes, int32_t* idx_out, float* out,
+                                        cudaStream_t stream);
+
+/*
+ * Paged caches (block tables, the layout of paged-attention serving engines).  A
+ * pool of num_pages pages, each holding page_size consecutive positions of every
+ * kv head: k_pages, v_pages [num_pages][Hkv][page_size][d] elements of `dt`,
+ * code_pages [num_pages][Hkv][page_size][d/4] bytes (adamas_encode_pages).
+ * Position p of sequence b lives in page block_table[b * max_blocks_per_seq +
+ * p / page_size], row p % page_size.  page_size is a power of two in [1, 2^20];
+ * max_blocks_per_seq * page_size >= max_seq_len; seq_lens [B] int32 in
+ * [0, max_seq_len] (device).  Entries of a block-table row past the sequence's
+ * last page are never read.  The kernel copies each page's codes straight into
+ * shared memory and gathers the selected K/V rows through the table.  idx_out,
+ * out, shared and the error behaviour are those of adamas_decode_step_varlen with
+ * Lmax = max_seq_len; a page id outside [0, num_pages) is read on the device: page
+ * 0 is used instead and the error word records it (ADAMAS_ERR_INVALID_ARG).
+ */
+adamas_status adamas_decode_step_paged(const void* q, const void* k_pages, const void* v_pages,
+                                       const uint8_t* code_pages, adamas_dtype dt, int B, int Hq,
+                                       int Hkv, int d, int page_size, int64_t num_pages,
+                                       const int32_t* block_table, int max_blocks_per_seq,
+                                       const int32_t* seq_lens, int64_t max_seq_len, int k,
+                                       float t, int shared, void* workspace, size_t ws_bytes,
+                                       int32_t* idx_out, float* out, cudaStream_t stream);
+
+/* Stage entry point: distance scan + top-k over paged codes from query codes. */
+adamas_status adamas_select_topk_paged(const uint8_t* qcodes, const uint8_t* code_pages, int B,
+                                       int Hq, int Hkv, int page_size, int64_t num_pages,
+                                       const int32_t* block_table, int max_blocks_per_seq,
+                                       const int32_t* seq_lens, int64_t max_seq_len, int k,
+                                       int shared, void* workspace, size_t ws_bytes,
+                                       int32_t* idx_out, cudaStream_t stream);
+
+/*
+ * Key encoder for paged caches: encodes every row (all kv heads, all page_size
+ * positions) of the pages page_ids[0 .. n_ids) of k_pages into code_pages (layouts
+ * as in adamas_decode_step_paged); page_ids == NULL encodes all num_pages pages.
+ * Appending a token re-encodes its page.  Page ids outside [0, num_pages) are
+ * skipped.
+ */
+adamas_status adamas_encode_pages(const void* k_pages, adamas_dtype dt, int Hkv, int d,
+                                  int page_size, int64_t num_pages, const int32_t* page_ids,
+                                  int64_t n_ids, float t, uint8_t* code_pages,
+                                  cudaStream_t stream);
 
 /* Workspace of adamas_sparse_attention, in bytes (zero-filled once, self-cleaning). */
 size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff);

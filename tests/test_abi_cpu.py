@@ -141,3 +141,60 @@ def test_shared_entry_points_reject_and_plan():
         assert q["tokens_per_cta"] * q["cluster"] >= L and q["tokens_per_cta"] <= 65535
         assert q["smem_bytes"] <= 232448
     assert ad.decode_plan_shared(1, 32, 8, 32768, 128)["cluster"] == 16
+
+
+def test_varlen_and_paged_entry_points_reject():
+    v = ad.lib().adamas_decode_step_varlen
+    ok = [A, A, A, A, BF16, 2, 32, 8, 128, 4096, A, 128, 1.0, 0, A, 1 << 30, None, A, None]
+    for i, bad in [(10, None), (10, A + 2), (13, 2), (0, None), (8, 64), (9, 0)]:
+        args = list(ok); args[i] = bad
+        want = ERR_UNSUPPORTED if i == 8 else ERR_INVALID_ARG
+        assert v(*args) == want, (i, bad)
+    p = ad.lib().adamas_decode_step_paged
+    ok = [A, A, A, A, BF16, 2, 32, 8, 128, 16, 100, A, 64, A, 1024, 128, 1.0, 0, A, 1 << 30, None,
+          A, None]
+    cases = [
+        (9, 24),        # page size not a power of two
+        (9, 0),
+        (9, 1 << 21),   # page size above 2^20
+        (10, 0),        # no pages
+        (11, None),     # no block table
+        (13, None),     # no lengths
+        (12, 63),       # 63 blocks x 16 < 1024 positions
+        (14, 0),
+        (17, 5),        # shared flag not 0/1
+        (11, A + 2),    # misaligned table
+    ]
+    for i, bad in cases:
+        args = list(ok); args[i] = bad
+        assert p(*args) == ERR_INVALID_ARG, (i, bad)
+    args = list(ok); args[8] = 96
+    assert p(*args) == ERR_UNSUPPORTED
+    s = ad.lib().adamas_select_topk_paged
+    assert s(None, A, 2, 32, 8, 16, 100, A, 64, A, 1024, 128, 0, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    assert s(A, A, 2, 32, 8, 16, 100, A, 64, A, 1024, 128, 0, A, 1 << 30, None, None) == ERR_INVALID_ARG
+    e = ad.lib().adamas_encode_pages
+    assert e(None, BF16, 8, 128, 16, 100, None, 0, 1.0, A, None) == ERR_INVALID_ARG
+    assert e(A, BF16, 8, 64, 16, 100, None, 0, 1.0, A, None) == ERR_UNSUPPORTED
+    assert e(A, BF16, 8, 128, 16, 0, None, 0, 1.0, A, None) == ERR_INVALID_ARG
+    assert e(A, BF16, 8, 128, 16, 100, A, -1, 1.0, A, None) == ERR_INVALID_ARG
+
+
+def test_paging_helper_layout():
+    """workloads.paging puts position p of sequence b at page table[b, p // page], row
+    p % page, with distinct pages per block and spare pages left at the fill value."""
+    import torch
+    from workloads.paging import make_block_table, scatter_to_pages
+    lens = [37, 0, 16]
+    pc = make_block_table(lens, 40, 16, seed=3, spare=2)
+    assert pc.num_pages == 3 + 0 + 1 + 2
+    used = pc.block_table[pc.block_table >= 0].tolist()
+    assert len(used) == len(set(used)) == 4
+    x = torch.arange(3 * 2 * 40, dtype=torch.float32).reshape(3, 2, 40, 1)
+    pool = scatter_to_pages(x, pc, fill=-1)
+    for b, L in enumerate(lens):
+        for p in range(L):
+            page = int(pc.block_table[b, p // 16])
+            assert torch.equal(pool[page, :, p % 16], x[b, :, p])
+    spare = set(range(pc.num_pages)) - set(used)
+    assert all((pool[s] == -1).all() for s in spare)

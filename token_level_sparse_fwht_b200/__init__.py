@@ -60,6 +60,16 @@ _SIGNATURES = {
                                               _c_sz, _c_p, _c_p, _c_p, _c_p]),
     "adamas_select_topk_shared": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i,
                                          _c_p, _c_sz, _c_p, _c_p]),
+    "adamas_decode_step_varlen": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                         _c_i64, _c_p, _c_i, _c_f, _c_i, _c_p, _c_sz, _c_p, _c_p,
+                                         _c_p]),
+    "adamas_decode_step_paged": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                        _c_i, _c_i64, _c_p, _c_i, _c_p, _c_i64, _c_i, _c_f, _c_i,
+                                        _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "adamas_select_topk_paged": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_p, _c_i,
+                                        _c_p, _c_i64, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "adamas_encode_pages": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_p, _c_i64, _c_f,
+                                   _c_p, _c_p]),
     "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "adamas_sparse_attention": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i, _c_i,
                                        _c_i64, _c_i, _c_p, _c_sz, _c_p, _c_p]),
@@ -314,6 +324,78 @@ def select_topk(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
 def select_topk_shared(qcodes, codes, L: int, k: int, ws, idx_out=None, stream=None):
     """Shared selection from query codes: idx [B,Hkv,min(k,L)] int32."""
     return _select("adamas_select_topk_shared", "Hkv", qcodes, codes, L, k, ws, idx_out, stream)
+
+
+# ------------------------------------ per-sequence lengths and paged caches
+def _i32(t: torch.Tensor, name: str):
+    if t.dtype != torch.int32:
+        raise TypeError(f"{name} must be int32")
+    return _dev(t, name)
+
+
+def decode_step_varlen(q, k_cache, v_cache, codes, seq_lens, k: int, t: float, ws,
+                       shared: bool = False, idx_out=None, out=None, stream=None):
+    """Decode step with per-sequence lengths seq_lens [B] int32 (device) over
+    contiguous caches [B,Hkv,Lmax,128].  Returns out [B,Hq,128]; idx_out, if given,
+    is [B, Hq (Hkv if shared), min(k, Lmax)] int32, -1 past a sequence's count."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
+    _check(lib().adamas_decode_step_varlen(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(codes, "codes"),
+        _dtype_code(k_cache), B, Hq, Hkv, d, Lmax, _i32(seq_lens, "seq_lens"), k, float(t),
+        int(bool(shared)), _dev(ws, "workspace"), ws.numel(), idx_ptr, _dev(out, "out"),
+        _stream(stream)), "adamas_decode_step_varlen")
+    return out
+
+
+def decode_step_paged(q, k_pages, v_pages, code_pages, block_table, seq_lens,
+                      max_seq_len: int, k: int, t: float, ws, shared: bool = False,
+                      idx_out=None, out=None, stream=None):
+    """Decode step over paged caches: k_pages, v_pages [P,Hkv,page,128], code_pages
+    [P,Hkv,page,32], block_table [B,max_blocks] int32, seq_lens [B] int32."""
+    B, Hq, d = q.shape
+    P, Hkv, page, _ = k_pages.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
+    _check(lib().adamas_decode_step_paged(
+        _dev(q, "q"), _dev(k_pages, "k_pages"), _dev(v_pages, "v_pages"),
+        _dev(code_pages, "code_pages"), _dtype_code(k_pages), B, Hq, Hkv, d, page, P,
+        _i32(block_table, "block_table"), block_table.shape[1], _i32(seq_lens, "seq_lens"),
+        max_seq_len, k, float(t), int(bool(shared)), _dev(ws, "workspace"), ws.numel(), idx_ptr,
+        _dev(out, "out"), _stream(stream)), "adamas_decode_step_paged")
+    return out
+
+
+def select_topk_paged(qcodes, code_pages, block_table, seq_lens, max_seq_len: int, k: int, ws,
+                      shared: bool = False, idx_out=None, stream=None):
+    B, Hq, _ = qcodes.shape
+    P, Hkv, page, _ = code_pages.shape
+    if idx_out is None:
+        idx_out = torch.empty((B, Hkv if shared else Hq, min(k, max_seq_len)), dtype=torch.int32,
+                              device=qcodes.device)
+    _check(lib().adamas_select_topk_paged(
+        _dev(qcodes, "qcodes"), _dev(code_pages, "code_pages"), B, Hq, Hkv, page, P,
+        _i32(block_table, "block_table"), block_table.shape[1], _i32(seq_lens, "seq_lens"),
+        max_seq_len, k, int(bool(shared)), _dev(ws, "workspace"), ws.numel(),
+        _dev(idx_out, "idx_out"), _stream(stream)), "adamas_select_topk_paged")
+    return idx_out
+
+
+def encode_pages(k_pages, code_pages, t: float, page_ids=None, stream=None):
+    """Encodes all rows of the listed pages (int32 device tensor; None: every page)."""
+    P, Hkv, page, d = k_pages.shape
+    if code_pages.dtype != torch.uint8 or tuple(code_pages.shape) != (P, Hkv, page, d // 4):
+        raise ValueError("code_pages must be uint8 [P, Hkv, page, d/4]")
+    ids = None if page_ids is None else _i32(page_ids, "page_ids")
+    n = 0 if page_ids is None else page_ids.numel()
+    _check(lib().adamas_encode_pages(_dev(k_pages, "k_pages"), _dtype_code(k_pages), Hkv, d, page,
+                                     P, ids, n, float(t), _dev(code_pages, "code_pages"),
+                                     _stream(stream)), "adamas_encode_pages")
+    return code_pages
 
 
 def sparse_attention_workspace(B: int, Hq: int, k_eff: int, device="cuda", stream=None):

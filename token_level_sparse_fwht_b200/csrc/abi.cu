@@ -40,6 +40,12 @@ bool good_group(int Hq, int Hkv) {
 }
 adamas_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ADAMAS_OK : ADAMAS_ERR_CUDA; }
 
+CacheLayout contiguous(int64_t Lmax) {
+  CacheLayout c;
+  c.Lmax = Lmax;
+  return c;
+}
+
 // Device address of a page-locked, device-mapped host buffer; nullptr for any
 // other memory (pageable host memory, device memory, unknown pointers).
 template <typename P>
@@ -123,6 +129,7 @@ adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream
     return ADAMAS_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
   if (word & (kErrBarrier | kErrCopy)) return ADAMAS_ERR_TIMEOUT;
+  if (word & kErrInput) return ADAMAS_ERR_INVALID_ARG;
   return word ? ADAMAS_ERR_INTERNAL : ADAMAS_OK;
 }
 
@@ -137,7 +144,8 @@ adamas_status plan_common(bool shared, int B, int Hq, int Hkv, int d, int64_t L,
   const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, L, L, k);
   if (s != ADAMAS_OK) return s;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
   if (ctas) *ctas = p.grid;
   if (cluster) *cluster = p.cluster;
   if (tokens_per_cta) *tokens_per_cta = p.keys_per_cta;
@@ -158,10 +166,12 @@ adamas_status decode_common(bool shared, const void* q, const void* k_cache,
       !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
-  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv, Lmax, L,
-                                 k, t, workspace, idx_out, out, shared, p, stream));
+  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
+                                 contiguous(Lmax), L, k, t, workspace, idx_out, out, shared, p,
+                                 stream));
 }
 
 adamas_status decode_host_common(bool shared, const void* q_host, void* q_dev,
@@ -182,7 +192,8 @@ adamas_status decode_host_common(bool shared, const void* q_host, void* q_dev,
       (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   // Page-locked host buffers are mapped into the device's address space: then the
   // kernel reads q from, and writes out to, host memory itself (no copy engines,
@@ -191,8 +202,8 @@ adamas_status decode_host_common(bool shared, const void* q_host, void* q_dev,
   void* oh_dev = mapped_device_pointer(out_host);
   if (qh_dev && oh_dev && aligned(qh_dev, 16) && aligned(oh_dev, 16)) {
     return from_cuda(launch_decode(qh_dev, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
-                                   Lmax, L, k, t, workspace, idx_out, static_cast<float*>(oh_dev),
-                                   shared, p, stream));
+                                   contiguous(Lmax), L, k, t, workspace, idx_out,
+                                   static_cast<float*>(oh_dev), shared, p, stream));
   }
   const size_t elem = dt == ADAMAS_F32 ? 4 : 2;
   const size_t qbytes = size_t(B) * Hq * kD * elem;
@@ -200,8 +211,8 @@ adamas_status decode_host_common(bool shared, const void* q_host, void* q_dev,
   if (cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return ADAMAS_ERR_CUDA;
   const adamas_status r = from_cuda(launch_decode(q_dev, nullptr, k_cache, v_cache, codes, dt, B,
-                                                  Hq, Hkv, Lmax, L, k, t, workspace, idx_out,
-                                                  out_dev, shared, p, stream));
+                                                  Hq, Hkv, contiguous(Lmax), L, k, t, workspace,
+                                                  idx_out, out_dev, shared, p, stream));
   if (r != ADAMAS_OK) return r;
   return from_cuda(cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, stream));
 }
@@ -216,11 +227,59 @@ adamas_status select_common(bool shared, const uint8_t* qcodes, const uint8_t* c
       !aligned(idx_out, 4))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, p)) return ADAMAS_ERR_UNSUPPORTED;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(nullptr, qcodes, nullptr, nullptr, codes, ADAMAS_BF16, B, Hq,
-                                 Hkv, Lmax, L, k, 0.0f, workspace, idx_out, nullptr, shared, p,
-                                 stream));
+                                 Hkv, contiguous(Lmax), L, k, 0.0f, workspace, idx_out, nullptr,
+                                 shared, p, stream));
+}
+
+// Checks of the page-pool arguments shared by the paged entry points; fills `lay`.
+adamas_status check_pages(int page_size, int64_t num_pages, const int32_t* block_table,
+                          int max_blocks, const int32_t* seq_lens, int64_t max_seq_len,
+                          CacheLayout& lay) {
+  if (!block_table || !seq_lens) return ADAMAS_ERR_INVALID_ARG;
+  if (page_size < 1 || page_size > (1 << 20) || (page_size & (page_size - 1)))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (num_pages < 1 || num_pages > INT32_MAX || max_blocks < 1 || max_seq_len < 1)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (int64_t(max_blocks) * page_size < max_seq_len) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(block_table, 4) || !aligned(seq_lens, 4)) return ADAMAS_ERR_INVALID_ARG;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  lay.block_table = block_table;
+  lay.max_blocks = max_blocks;
+  lay.page_shift = shift;
+  lay.num_pages = num_pages;
+  lay.seq_lens = seq_lens;
+  return ADAMAS_OK;
+}
+
+// Decode or select (q == nullptr: from qcodes, no attention) over any cache layout.
+adamas_status layout_common(bool shared, const void* q, const uint8_t* qcodes, const void* kc,
+                            const void* vc, const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                            int Hkv, int d, const CacheLayout& lay, int64_t L, int k, float t,
+                            void* workspace, size_t ws_bytes, int32_t* idx_out, float* out,
+                            cudaStream_t stream) {
+  const bool select_only = q == nullptr;
+  if (!codes || !workspace) return ADAMAS_ERR_INVALID_ARG;
+  if (select_only ? (!qcodes || !idx_out) : (!kc || !vc || !out)) return ADAMAS_ERR_INVALID_ARG;
+  if (!select_only && (!good_dtype(dt) || !good_t(t))) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, L, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(codes, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (select_only ? !aligned(qcodes, 16)
+                  : (!aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(out, 16)))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  const int page_shift = lay.block_table != nullptr ? lay.page_shift : -1;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, page_shift, p))
+    return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_decode(q, qcodes, kc, vc, codes, select_only ? ADAMAS_BF16 : dt, B, Hq,
+                                 Hkv, lay, L, k, t, workspace, idx_out, out, shared, p, stream));
 }
 
 }  // namespace
@@ -284,6 +343,68 @@ adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, in
                                  size_t ws_bytes, int32_t* idx_out, cudaStream_t stream) {
   return select_common(false, qcodes, codes, B, Hq, Hkv, Lmax, L, k, workspace, ws_bytes,
                        idx_out, stream);
+}
+
+adamas_status adamas_decode_step_varlen(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, const int32_t* seq_lens,
+                                        int k, float t, int shared, void* workspace,
+                                        size_t ws_bytes, int32_t* idx_out, float* out,
+                                        cudaStream_t stream) {
+  if (!q || !seq_lens || !aligned(seq_lens, 4) || (shared != 0 && shared != 1))
+    return ADAMAS_ERR_INVALID_ARG;
+  CacheLayout lay = contiguous(Lmax);
+  lay.seq_lens = seq_lens;
+  return layout_common(shared != 0, q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv, d, lay,
+                       Lmax, k, t, workspace, ws_bytes, idx_out, out, stream);
+}
+
+adamas_status adamas_decode_step_paged(const void* q, const void* k_pages, const void* v_pages,
+                                       const uint8_t* code_pages, adamas_dtype dt, int B, int Hq,
+                                       int Hkv, int d, int page_size, int64_t num_pages,
+                                       const int32_t* block_table, int max_blocks_per_seq,
+                                       const int32_t* seq_lens, int64_t max_seq_len, int k,
+                                       float t, int shared, void* workspace, size_t ws_bytes,
+                                       int32_t* idx_out, float* out, cudaStream_t stream) {
+  if (!q || (shared != 0 && shared != 1)) return ADAMAS_ERR_INVALID_ARG;
+  CacheLayout lay;
+  const adamas_status s = check_pages(page_size, num_pages, block_table, max_blocks_per_seq,
+                                      seq_lens, max_seq_len, lay);
+  if (s != ADAMAS_OK) return s;
+  return layout_common(shared != 0, q, nullptr, k_pages, v_pages, code_pages, dt, B, Hq, Hkv, d,
+                       lay, max_seq_len, k, t, workspace, ws_bytes, idx_out, out, stream);
+}
+
+adamas_status adamas_select_topk_paged(const uint8_t* qcodes, const uint8_t* code_pages, int B,
+                                       int Hq, int Hkv, int page_size, int64_t num_pages,
+                                       const int32_t* block_table, int max_blocks_per_seq,
+                                       const int32_t* seq_lens, int64_t max_seq_len, int k,
+                                       int shared, void* workspace, size_t ws_bytes,
+                                       int32_t* idx_out, cudaStream_t stream) {
+  if (!qcodes || (shared != 0 && shared != 1)) return ADAMAS_ERR_INVALID_ARG;
+  CacheLayout lay;
+  const adamas_status s = check_pages(page_size, num_pages, block_table, max_blocks_per_seq,
+                                      seq_lens, max_seq_len, lay);
+  if (s != ADAMAS_OK) return s;
+  return layout_common(shared != 0, nullptr, qcodes, nullptr, nullptr, code_pages, ADAMAS_BF16, B,
+                       Hq, Hkv, kD, lay, max_seq_len, k, 0.0f, workspace, ws_bytes, idx_out,
+                       nullptr, stream);
+}
+
+adamas_status adamas_encode_pages(const void* k_pages, adamas_dtype dt, int Hkv, int d,
+                                  int page_size, int64_t num_pages, const int32_t* page_ids,
+                                  int64_t n_ids, float t, uint8_t* code_pages,
+                                  cudaStream_t stream) {
+  if (!k_pages || !code_pages || !good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (Hkv <= 0 || page_size < 1 || num_pages < 1 || num_pages > INT32_MAX)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (page_ids && (n_ids < 0 || !aligned(page_ids, 4))) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(k_pages, 16) || !aligned(code_pages, 16)) return ADAMAS_ERR_INVALID_ARG;
+  const int64_t per = int64_t(Hkv) * page_size;           // rows per page
+  const int64_t groups = page_ids ? n_ids : num_pages;
+  return from_cuda(launch_encode_rows(k_pages, dt, code_pages, groups * per, per, per, 0, t,
+                                      stream, page_ids, num_pages));
 }
 
 adamas_status adamas_select_topk_shared(const uint8_t* qcodes, const uint8_t* codes, int B,

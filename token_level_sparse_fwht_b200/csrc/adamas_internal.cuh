@@ -19,6 +19,7 @@ constexpr int kPartStride = 132;        // m, l, 2 pad, acc[128] (floats)
 constexpr uint32_t kErrBarrier = 1u;
 constexpr uint32_t kErrCopy = 2u;
 constexpr uint32_t kErrSelect = 4u;   // top-k bookkeeping found no k-th distance
+constexpr uint32_t kErrInput = 8u;    // a device-resident length or page id out of range
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
 
 // ----------------------------------------------------------------- PTX helpers
@@ -57,6 +58,31 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           "r"(smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared (both 16-B aligned), completed by the
+// issuing thread's commit groups.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most `pending` (0..7) of this thread's commit groups are in flight.
+__device__ __forceinline__ void cp_async_wait_pending(int pending) {
+  switch (pending) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
@@ -458,17 +484,33 @@ struct Plan {
   int stages;            // bulk-copy ring depth
   size_t smem;           // dynamic shared memory bytes
 };
+// page_shift: log2(page size) for paged caches, -1 for contiguous caches.
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
-                                    Plan& p);
+                                    int page_shift, Plan& p);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k);
 size_t decode_workspace_error_offset();
+// Where a unit's positions live.  Contiguous caches: unit (b, kv head) owns rows
+// [unit * Lmax, unit * Lmax + L).  Paged caches (block_table != nullptr): position p
+// of sequence b is row p & (page - 1) of kv head h in page block_table[b][p >> shift],
+// pages laid out [page][Hkv][page size][...].  seq_lens (nullable) gives each
+// sequence its own length <= L.
+struct CacheLayout {
+  int64_t Lmax = 0;
+  const int32_t* seq_lens = nullptr;
+  const int32_t* block_table = nullptr;
+  int max_blocks = 0;
+  int page_shift = 0;
+  int64_t num_pages = 0;
+};
 cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
-                          int64_t Lmax, int64_t L, int kk, float t, void* ws, int32_t* idx_out,
-                          float* out, bool shared, const Plan& p, cudaStream_t stream);
+                          const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
+                          int32_t* idx_out, float* out, bool shared, const Plan& p,
+                          cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const int32_t* ids = nullptr,
+                               int64_t id_limit = 0);
 size_t attention_workspace_bytes(int B, int Hq, int k_eff);
 bool noalloc_fits(int B, int Hq);
 cudaError_t launch_sparse_attention_noalloc(const void* q, const void* k, const void* v,

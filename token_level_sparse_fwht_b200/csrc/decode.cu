@@ -51,15 +51,21 @@ __host__ __device__ inline int dist_stride(int R) { return (R + 7) & ~7; }
 struct DecodeArgs {
   const void* q;             // [B][Hq][128] (encode mode) or nullptr
   const uint8_t* qcodes;     // [B][Hq][32] (select mode) or nullptr
-  const void* k;             // [B][Hkv][Lmax][128]
+  const void* k;             // [B][Hkv][Lmax][128], or pages [P][Hkv][page][128]
   const void* v;
-  const uint8_t* codes;      // [B][Hkv][Lmax][32]
+  const uint8_t* codes;      // [B][Hkv][Lmax][32], or pages [P][Hkv][page][32]
   int B, Hq, Hkv;
-  int64_t Lmax, L;
-  int k_eff;
+  int64_t Lmax, L;           // cache rows per unit (contiguous layout); longest context
+  int budget;                // k; a unit selects min(k, its length) positions
+  int idx_stride;            // idx_out row length, min(k, L)
+  const int32_t* seq_lens;   // [B] context lengths, or nullptr (every sequence has L)
+  const int32_t* block_table;  // [B][max_blocks] page ids, or nullptr (contiguous)
+  int max_blocks;
+  int page_shift;            // log2(page size)
+  int64_t num_pages;
   float t;
   float scale_log2;
-  int32_t* idx_out;          // [B][Hq][k_eff] or nullptr
+  int32_t* idx_out;          // [B][rows][idx_stride] or nullptr (-1 past a unit's count)
   float* out;                // [B][Hq][128] or nullptr (select mode)
   uint32_t* err;             // device error word
   int cluster;               // CTAs per unit
@@ -89,7 +95,8 @@ static_assert(Sel<1, false>::NB == kNBins && Sel<1, false>::BS == kBinStride &&
 static_assert(Sel<8, true>::NB <= 0x7fff, "summed distances must fit a signed 16-bit lane");
 
 struct SmemLayout {
-  size_t ring, mbar, hist, coarse, fine, dist, list, qf, qc, qth, scan, merge, info, misc, total;
+  size_t ring, mbar, hist, coarse, fine, dist, list, qf, qc, qth, scan, merge, info, ptab, misc,
+      total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -99,7 +106,7 @@ __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / 
 // after the partials: the ring is idle once the scan is over, and rank 0 receives
 // the peers' partials only after the first cluster barrier.
 __host__ __device__ inline SmemLayout make_layout(int G, int GS, int BS, int FW, int GM, int R,
-                                                 int list_cap, int CS, int stages) {
+                                                 int list_cap, int CS, int stages, int ptab) {
   SmemLayout s;
   size_t o = 0;
   const size_t ring = size_t(stages) * kChunk * kCodeBytes;
@@ -122,15 +129,22 @@ __host__ __device__ inline SmemLayout make_layout(int G, int GS, int BS, int FW,
     s.merge = o; o = al(o + merge, 128);
   }
   s.info = o;  o = al(o + size_t(GS) * 9 * 4, 128);
+  s.ptab = o;  o = al(o + size_t(ptab) * 4, 128);   // page ids of the CTA's range (paged)
   s.misc = o;  o = al(o + 128, 128);
   s.total = o;
   return s;
 }
 
 template <int G, bool SH>
-__host__ __device__ inline SmemLayout layout_of(int R, int list_cap, int CS, int stages) {
+__host__ __device__ inline SmemLayout layout_of(int R, int list_cap, int CS, int stages,
+                                                int ptab) {
   using X = Sel<G, SH>;
-  return make_layout(G, X::GS, X::BS, X::FW, X::GM, R, list_cap, CS, stages);
+  return make_layout(G, X::GS, X::BS, X::FW, X::GM, R, list_cap, CS, stages, ptab);
+}
+
+// Page-table entries a CTA stages: the pages its R positions can span.
+__host__ __device__ inline int ptab_entries(int R, int page_shift, bool paged) {
+  return paged ? ((R + (1 << page_shift) - 1) >> page_shift) + 1 : 0;
 }
 
 // Bit 15 and bit 31 of w0, then of w1, as bits 0..3 (the sign bits of four packed
@@ -183,7 +197,7 @@ __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t 
   }
 }
 
-template <int G, bool SH, typename T>
+template <int G, bool SH, bool PG, typename T>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a) {
   using X = Sel<G, SH>;
   constexpr int GS = X::GS, BS = X::BS, NB = X::NB, CB = X::C, FW = X::FW, GM = X::GM;
@@ -192,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   const int CS = a.cluster;
   const int rank = int(cluster.block_rank());
   const int S = a.stages;
-  const SmemLayout lo = layout_of<G, SH>(a.keys_per_cta, a.list_cap, CS, S);
+  const SmemLayout lo = layout_of<G, SH>(a.keys_per_cta, a.list_cap, CS, S,
+                                         ptab_entries(a.keys_per_cta, a.page_shift, PG));
   uint8_t* ring = smem + lo.ring;
   float* part = reinterpret_cast<float*>(smem + lo.ring);           // [CS][G][kPartStride]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
@@ -207,28 +222,110 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   uint32_t* scan = reinterpret_cast<uint32_t*>(smem + lo.scan);    // [2][kWarps][GS]
   float* merge = reinterpret_cast<float*>(smem + lo.merge);        // [kWarps][GM][kPartStride]
   int* info = reinterpret_cast<int*>(smem + lo.info);              // [GS][8], then [GS]
+  int32_t* ptab = reinterpret_cast<int32_t*>(smem + lo.ptab);      // paged: row bases
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int unit = blockIdx.x / CS;
   const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int64_t L = a.L;
+  // this unit's context length (a length outside [0, L] is an input error: flagged,
+  // clamped) and the number of positions it selects
+  int64_t L = a.L;
+  if (a.seq_lens != nullptr) {
+    const int64_t Lb = a.seq_lens[b];
+    if (Lb < 0 || Lb > a.L) {
+      if (tid == 0) atomicOr(a.err, kErrInput);
+    }
+    L = min(max(Lb, int64_t(0)), a.L);
+  }
+  const int keff = int(min(int64_t(a.budget), L));
   const int R = a.keys_per_cta;
   const int RS = dist_stride(R);
   const int64_t p0 = int64_t(rank) * R;
   const int n = int(max(int64_t(0), min(int64_t(R), L - p0)));   // keys of this CTA
   const int nch = (n + kChunk - 1) / kChunk;
   const uint8_t* codes = a.codes + (int64_t(unit) * a.Lmax + p0) * kCodeBytes;
+  // paged caches: position p of this unit lives in page block_table[b][p >> shift]
+  // (rows [page][kv head][p & mask]).  The last warp stages, for every page of this
+  // CTA's range, the row of its first position for this kv head in shared memory
+  // (pool rows number below 2^31: a row is at least 256 bytes); a page id outside
+  // [0, num_pages) is an input error: flagged, and page 0 is used instead so that no
+  // access leaves the pool.
+  constexpr bool paged = PG;
+  const int psh = a.page_shift;
+  const int pmask = (1 << psh) - 1;
+  const int64_t pfirst = p0 >> psh;
+  // row of position p in the K/V (and code) storage
+  const auto row_of = [&](int64_t p) -> int64_t {
+    if constexpr (!paged) {
+      return int64_t(unit) * a.Lmax + p;
+    } else {
+      return int64_t(ptab[(p >> psh) - pfirst] + (int(p) & pmask));
+    }
+  };
+  // chunk qi of this CTA's codes into ring slot `slot`.  Contiguous caches: one
+  // bulk copy on the slot's mbarrier, issued by one thread.  Paged caches: each warp
+  // copies the 32 keys its threads scan (1 KB) with 16-byte asynchronous copies, one
+  // commit group per chunk: lanes 2m, 2m + 1 take the two halves of key m (then of
+  // key m + 16), so each instruction reads 512 contiguous bytes of a page, and a
+  // page of any size costs no extra copy instruction.
+  const auto issue_chunk = [&](int qi, int slot) {
+    if constexpr (!paged) {
+      const int c0 = qi * kChunk;
+      const int keys = min(kChunk, n - c0);
+      mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes));
+      bulk_g2s(ring + size_t(slot) * kChunk * kCodeBytes, codes + int64_t(c0) * kCodeBytes,
+               uint32_t(keys * kCodeBytes), &mbar[slot]);
+    } else {
+      // positions and rows fit 32 bits (a CTA range starts below 2^20; pool rows
+      // number below 2^31)
+      const int kk = warp * 32 + (lane >> 1);       // key of this lane's first half
+      const int half = (lane & 1) * 16;
+      uint8_t* dst = ring + (slot * kChunk + kk) * kCodeBytes + half;
+      const int r = qi * kChunk + kk;
+      const int pos = int(p0) + r;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {               // keys kk and kk + 16
+        if (qi < nch && r + 16 * i < n) {
+          const int pi = pos + 16 * i;
+          const int row = ptab[(pi >> psh) - int(pfirst)] + (pi & pmask);
+          cp_async_16(dst + 16 * i * kCodeBytes, a.codes + int64_t(row) * kCodeBytes + half);
+        }
+      }
+      cp_async_commit();
+    }
+  };
 
   // ---- issue the code copies first: HBM traffic starts before anything else.  The
   // last warp issues them, so the warps that encode the queries are not delayed.
-  if (tid == kThreads - 32) {
-    for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
-    fence_mbar_init();
-    for (int qi = 0; qi < min(nch, S); ++qi) {
-      const int keys = min(kChunk, n - qi * kChunk);
-      mbar_expect_tx(&mbar[qi], uint32_t(keys * kCodeBytes));
-      bulk_g2s(ring + size_t(qi) * kChunk * kCodeBytes,
-               codes + int64_t(qi) * kChunk * kCodeBytes, uint32_t(keys * kCodeBytes), &mbar[qi]);
+  if constexpr (!paged) {
+    if (tid == kThreads - 32) {
+      for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
+      fence_mbar_init();
+      for (int qi = 0; qi < min(nch, S); ++qi) issue_chunk(qi, qi);
+    }
+  } else {
+    // paged: the whole block stages the page table, four independent loads in
+    // flight per thread (the copies start after the prologue's barrier)
+    const int32_t* bt = a.block_table + int64_t(b) * a.max_blocks + pfirst;
+    const int npages = n > 0 ? int(((p0 + n - 1) >> psh) - pfirst + 1) : 0;
+    for (int i0 = tid; i0 < npages; i0 += 4 * kThreads) {
+      int32_t pg[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kThreads;
+        pg[u] = i < npages ? bt[i] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < npages) {
+          if (pg[u] < 0 || int64_t(pg[u]) >= a.num_pages) {
+            atomicOr(a.err, kErrInput);
+            pg[u] = 0;
+          }
+          ptab[i] = int32_t((int64_t(pg[u]) * a.Hkv + kvh) << psh);
+        }
+      }
     }
   }
 
@@ -247,6 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     }
   }
   __syncthreads();
+  if constexpr (paged) {
+    // page table staged: every thread starts its copies of the first S chunks (one
+    // commit group each, empty past the CTA's last chunk)
+    for (int qi = 0; qi < S; ++qi) issue_chunk(qi, qi);
+  }
   if (tid < G) {
     const uint32_t* wq = reinterpret_cast<const uint32_t*>(qc + tid * kCodeBytes);
     uint32_t wd[8];
@@ -281,7 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     int slot = 0;
     uint32_t parity = 0;
     for (int qi = 0; qi < nch; ++qi) {
-      mbar_wait_bounded(&mbar[slot], parity, a.err);
+      if constexpr (paged) {
+        cp_async_wait_pending(S - 1);   // this thread's copies of chunk qi have landed
+        __syncwarp();                   // ... and its warp-mates' (the key it scans)
+      } else {
+        mbar_wait_bounded(&mbar[slot], parity, a.err);
+      }
       const int r = qi * kChunk + tid;
       if (r < n) {
         const uint4* src = reinterpret_cast<const uint4*>(
@@ -320,16 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           atomicAdd(&hist[dsum], 1u);
         }
       }
-      // a slot is refilled only when the CTA's keys need more chunks than the ring
-      // holds; otherwise every chunk has its own slot and warps run ahead freely
-      if (nch > S) __syncthreads();
-      if (tid == kThreads - 32 && qi + S < nch) {
-        const int nx = qi + S;
-        const int keys = min(kChunk, n - nx * kChunk);
-        mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes));
-        bulk_g2s(ring + size_t(slot) * kChunk * kCodeBytes,
-                 codes + int64_t(nx) * kChunk * kCodeBytes, uint32_t(keys * kCodeBytes),
-                 &mbar[slot]);
+      if constexpr (paged) {
+        // the slot's entries for this warp's keys: every lane has read its own key
+        __syncwarp();
+        issue_chunk(qi + S, slot);
+      } else {
+        // a slot is refilled only when the CTA's keys need more chunks than the ring
+        // holds; otherwise every chunk has its own slot and warps run ahead freely
+        if (nch > S) __syncthreads();
+        if (tid == kThreads - 32 && qi + S < nch) issue_chunk(qi + S, slot);
       }
       if (++slot == S) { slot = 0; parity ^= 1u; }
     }
@@ -427,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     if (lane < kNCoarse) {
       for (int cc = 0; cc < CS; ++cc) S1 += coarse[(cc * GS + g) * kCoarseRow + lane];
     }
-    const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < kNCoarse && S1 >= uint32_t(a.k_eff));
+    const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < kNCoarse && S1 >= uint32_t(keff));
     if (lane == 0) jst[g] = __ffs(hit1) - 1;   // exists: chunk 29 ends at the last bin, count L
   }
   __syncthreads();
@@ -443,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   __syncthreads();
   if (warp < GS) {
     const int g = warp;
-    const uint32_t ke = uint32_t(a.k_eff);
+    const uint32_t ke = uint32_t(keff);
     const int jstar = jst[g];
     const int lo_bin = min(max(0, CB * jstar - 1) & ~3, BS - FW);
     // level 2, 32 bins per pass: lane l of pass p -> bin CB j* - 1 + 32 p + l.  The
@@ -559,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           while (m) {
             const int i = __ffs(m) - 1;
             m &= m - 1u;
-            const int64_t row_off = (int64_t(unit) * a.Lmax + p0 + s0 + i) * kD;
+            const int64_t row_off = row_of(p0 + s0 + i) * kD;
             prefetch_row_l2(static_cast<const T*>(a.k) + row_off);
             prefetch_row_l2(static_cast<const T*>(a.v) + row_off);
           }
@@ -582,7 +688,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         int rk = lt_b + min(eq_b, take[g]);
         // idx_out rows: [B][Hq] for per-head selection, [B][Hkv] for shared selection
         const int64_t orow_id = SH ? int64_t(b) * a.Hkv + kvh : int64_t(b) * a.Hq + kvh * G + g;
-        int32_t* orow = a.idx_out != nullptr ? a.idx_out + orow_id * a.k_eff + base[g] : nullptr;
+        int32_t* orow =
+            a.idx_out != nullptr ? a.idx_out + orow_id * a.idx_stride + base[g] : nullptr;
         uint16_t* lrow = list + size_t(g) * a.list_cap;
         while (sel) {
           const int i = __ffs(sel) - 1;
@@ -590,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           const int r = s0 + i;
           // rk < nsel and base + rk < k_eff hold by construction; the guard keeps a
           // broken invariant from writing outside the list or the output row
-          if (rk < nsel[g] && base[g] + rk < a.k_eff) {
+          if (rk < nsel[g] && base[g] + rk < keff) {
             lrow[rk] = static_cast<uint16_t>(r);
             if (orow) orow[rk] = int32_t(p0 + r);
           }
@@ -599,6 +706,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         carry_lt[g] += tot[g] >> 16;
         carry_eq[g] += tot[g] & 0xffffu;
       }
+    }
+  }
+  // a sequence shorter than the budget fills only keff slots of its rows: rank 0
+  // marks the rest -1
+  if (a.seq_lens != nullptr && a.idx_out != nullptr && rank == 0 && keff < a.idx_stride) {
+    const int pad = a.idx_stride - keff;
+    for (int i = tid; i < GS * pad; i += kThreads) {
+      const int g = i / pad;
+      const int64_t orow_id = SH ? int64_t(b) * a.Hkv + kvh : int64_t(b) * a.Hq + kvh * G + g;
+      a.idx_out[orow_id * a.idx_stride + keff + i % pad] = -1;
     }
   }
   __syncthreads();
@@ -616,8 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     const int sel_head = SH ? 0 : gi;
     const int nsel = info[sel_head * 8 + 3];
     const uint16_t* lrow = list + size_t(sel_head) * a.list_cap;
-    const T* kb = static_cast<const T*>(a.k) + int64_t(unit) * a.Lmax * kD;
-    const T* vb = static_cast<const T*>(a.v) + int64_t(unit) * a.Lmax * kD;
+    // contiguous caches: rows relative to the unit's base; paged: absolute pool rows
+    const int64_t base_row = paged ? 0 : int64_t(unit) * a.Lmax;
+    const T* kb = static_cast<const T*>(a.k) + base_row * kD;
+    const T* vb = static_cast<const T*>(a.v) + base_row * kD;
     float qv[GM][4];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
@@ -627,7 +746,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     SoftmaxState st[GM];
 #pragma unroll
     for (int h = 0; h < GM; ++h) st[h].init();
-    const auto pos_of = [&](int j) { return p0 + int64_t(lrow[j]); };
+    const auto pos_of = [&](int j) {
+      if constexpr (paged) {
+        return row_of(p0 + int64_t(lrow[j]));
+      } else {
+        return p0 + int64_t(lrow[j]);
+      }
+    };
     if constexpr (GM == 1) {
       attend_rows<T>(kb, vb, nsel, sub, WPG, pos_of, qv[0], a.scale_log2, lane, st[0]);
     } else {
@@ -665,6 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       const int gg = i / kD, dim = i % kD;
       float M = -INFINITY;
       for (int cc = 0; cc < CS; ++cc) M = fmaxf(M, part[(cc * G + gg) * kPartStride]);
+      if (M == -INFINITY) M = 0.f;   // every split empty (length 0): all terms below are 0
       float Ls = 0.f, A = 0.f;
       for (int cc = 0; cc < CS; ++cc) {
         const float* prow = part + (cc * G + gg) * kPartStride;
@@ -672,7 +798,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         Ls = fmaf(prow[1], e, Ls);
         A = fmaf(prow[4 + dim], e, A);
       }
-      a.out[(int64_t(b) * a.Hq + kvh * G + gg) * kD + dim] = A / Ls;
+      // an empty sequence (length 0) selects nothing: its output is zero
+      a.out[(int64_t(b) * a.Hq + kvh * G + gg) * kD + dim] = Ls > 0.f ? A / Ls : 0.f;
     }
   }
 }
@@ -687,17 +814,17 @@ static int max_smem_optin(int dev) {
   return v;
 }
 
-template <int G, bool SH, typename T>
+template <int G, bool SH, bool PG, typename T>
 static cudaError_t prepare_kernel() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     int dev = 0;
     cudaGetDevice(&dev);
-    err = cudaFuncSetAttribute(decode_kernel<G, SH, T>,
+    err = cudaFuncSetAttribute(decode_kernel<G, SH, PG, T>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem_optin(dev));
     if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(decode_kernel<G, SH, T>,
+      err = cudaFuncSetAttribute(decode_kernel<G, SH, PG, T>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   });
   return err;
@@ -705,7 +832,7 @@ static cudaError_t prepare_kernel() {
 
 template <int G, bool SH, typename T>
 static int active_clusters_g(int cs, size_t smem) {
-  if (prepare_kernel<G, SH, T>() != cudaSuccess) return 0;
+  if (prepare_kernel<G, SH, false, T>() != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs);
   cfg.blockDim = dim3(kThreads);
@@ -718,7 +845,7 @@ static int active_clusters_g(int cs, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int nclusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, SH, T>, &cfg) !=
+  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, SH, false, T>, &cfg) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -741,11 +868,12 @@ static int active_clusters(int G, bool shared, int cs, size_t smem) {
   return shared ? active_clusters_s<true>(G, cs, smem) : active_clusters_s<false>(G, cs, smem);
 }
 
-static size_t layout_total(int G, bool shared, int R, int list_cap, int cs, int stages) {
+static size_t layout_total(int G, bool shared, int R, int list_cap, int cs, int stages,
+                           int ptab) {
 #define ADAMAS_LAYOUT_CASE(GG)                                                        \
   case GG:                                                                            \
-    return shared ? layout_of<GG, true>(R, list_cap, cs, stages).total                \
-                  : layout_of<GG, false>(R, list_cap, cs, stages).total;
+    return shared ? layout_of<GG, true>(R, list_cap, cs, stages, ptab).total          \
+                  : layout_of<GG, false>(R, list_cap, cs, stages, ptab).total;
   switch (G) {
     ADAMAS_LAYOUT_CASE(1)
     ADAMAS_LAYOUT_CASE(2)
@@ -759,8 +887,8 @@ static size_t layout_total(int G, bool shared, int R, int list_cap, int cs, int 
 // Chooses the cluster size: among sizes whose shared memory fits (and, on a device,
 // whose clusters can be scheduled), the one with the least modelled time
 // waves x (per-key scan cost x keys per CTA + fixed per-wave latency).
-bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int sms,
-                      int smem_cap, bool query_device, Plan& p) {
+bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int page_shift,
+                      int sms, int smem_cap, bool query_device, Plan& p) {
   const int G = Hq / Hkv;
   const int64_t U = int64_t(B) * Hkv;
   const int64_t k_eff = std::min<int64_t>(k, L);
@@ -773,9 +901,11 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
     const int list_cap = int(std::max<int64_t>(1, std::min<int64_t>(R, k_eff)));
     const int64_t nchunks = (R + kChunk - 1) / kChunk;
     int stages = int(std::min<int64_t>(kMaxStages, std::max<int64_t>(1, nchunks)));
-    while (stages > 1 && layout_total(G, shared, int(R), list_cap, cs, stages) > size_t(smem_cap))
+    const int ptab = ptab_entries(int(R), page_shift, page_shift >= 0);
+    while (stages > 1 &&
+           layout_total(G, shared, int(R), list_cap, cs, stages, ptab) > size_t(smem_cap))
       --stages;
-    const size_t smem = layout_total(G, shared, int(R), list_cap, cs, stages);
+    const size_t smem = layout_total(G, shared, int(R), list_cap, cs, stages, ptab);
     if (smem > size_t(smem_cap)) continue;
     int conc_clusters = sms / cs;
     if (query_device) conc_clusters = active_clusters(G, shared, cs, smem);
@@ -801,23 +931,24 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
 }
 
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
-                                    Plan& p) {
+                                    int page_shift, Plan& p) {
   int dev = 0;
   const int sms = current_device_sms(&dev);
   if (sms <= 0) {
     // no device visible: plan for a 148-SM part with the sm_100 shared-memory cap
-    return make_decode_plan(B, Hq, Hkv, L, k, shared, 148, 232448, false, p);
+    return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, 148, 232448, false, p);
   }
-  return make_decode_plan(B, Hq, Hkv, L, k, shared, sms, max_smem_optin(dev), true, p);
+  return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, sms, max_smem_optin(dev), true,
+                          p);
 }
 
 // The decode workspace only carries the device error word (bounded copy waits).
 size_t decode_workspace_bytes(int, int, int, int64_t, int) { return 256; }
 size_t decode_workspace_error_offset() { return 8; }
 
-template <int G, bool SH, typename T>
+template <int G, bool SH, bool PG, typename T>
 static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t stream) {
-  const cudaError_t e = prepare_kernel<G, SH, T>();
+  const cudaError_t e = prepare_kernel<G, SH, PG, T>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
@@ -831,30 +962,43 @@ static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t str
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<G, SH, T>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<G, SH, PG, T>, a);
 }
 
-template <bool SH, typename T>
+template <bool SH, bool PG, typename T>
 static cudaError_t launch_t(int G, const DecodeArgs& a, const Plan& p, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_g<1, SH, T>(a, p, s);
-    case 2: return launch_g<2, SH, T>(a, p, s);
-    case 4: return launch_g<4, SH, T>(a, p, s);
-    case 8: return launch_g<8, SH, T>(a, p, s);
+    case 1: return launch_g<1, SH, PG, T>(a, p, s);
+    case 2: return launch_g<2, SH, PG, T>(a, p, s);
+    case 4: return launch_g<4, SH, PG, T>(a, p, s);
+    case 8: return launch_g<8, SH, PG, T>(a, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
+template <bool SH, bool PG>
+static cudaError_t launch_dt(adamas_dtype dt, int G, const DecodeArgs& a, const Plan& p,
+                             cudaStream_t s) {
+  if (dt == ADAMAS_F32) return launch_t<SH, PG, float>(G, a, p, s);
+  return launch_t<SH, PG, __nv_bfloat16>(G, a, p, s);
+}
+
 cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
-                          int64_t Lmax, int64_t L, int kk, float t, void* ws,
+                          const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
                           int32_t* idx_out, float* out, bool shared, const Plan& p,
                           cudaStream_t stream) {
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q; a.qcodes = qcodes; a.k = k; a.v = v; a.codes = codes;
-  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lmax = Lmax; a.L = L;
-  a.k_eff = int(std::min<int64_t>(kk, L));
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lmax = lay.Lmax; a.L = L;
+  a.budget = kk;
+  a.idx_stride = int(std::min<int64_t>(kk, L));
+  a.seq_lens = lay.seq_lens;
+  a.block_table = lay.block_table;
+  a.max_blocks = lay.max_blocks;
+  a.page_shift = lay.page_shift;
+  a.num_pages = lay.num_pages;
   a.t = t;
   a.scale_log2 = float(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   a.idx_out = idx_out; a.out = out;
@@ -864,12 +1008,13 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.list_cap = p.list_cap;
   a.stages = p.stages;
   a.attend = out != nullptr ? 1 : 0;
+  const bool paged = lay.block_table != nullptr;
   if (shared) {
-    if (dt == ADAMAS_F32) return launch_t<true, float>(G, a, p, stream);
-    return launch_t<true, __nv_bfloat16>(G, a, p, stream);
+    return paged ? launch_dt<true, true>(dt, G, a, p, stream)
+                 : launch_dt<true, false>(dt, G, a, p, stream);
   }
-  if (dt == ADAMAS_F32) return launch_t<false, float>(G, a, p, stream);
-  return launch_t<false, __nv_bfloat16>(G, a, p, stream);
+  return paged ? launch_dt<false, true>(dt, G, a, p, stream)
+               : launch_dt<false, false>(dt, G, a, p, stream);
 }
 
 }  // namespace adamas

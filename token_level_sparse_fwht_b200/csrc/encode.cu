@@ -10,29 +10,45 @@
 namespace adamas {
 
 // rows [nvec] of 128 elements: vector v lives at src + row_of(v) * 128 and its code
-// at dst + row_of(v) * 32, with row_of(v) = (v / per) * stride + off + v % per.
+// at dst + row_of(v) * 32, with row_of(v) = grp(v / per) * stride + off + v % per and
+// grp(i) = i, or ids[i] when a group list is given (groups whose id is outside
+// [0, id_limit) are skipped).
 template <typename T>
 __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ src,
                                                           uint8_t* __restrict__ dst,
                                                           int64_t nvec, int64_t per,
                                                           int64_t stride, int64_t off,
-                                                          float t) {
+                                                          float t,
+                                                          const int32_t* __restrict__ ids,
+                                                          int64_t id_limit) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   using R = Raw4<T>;
+  const auto row_of = [&](int64_t v, bool& ok) -> int64_t {
+    int64_t grp = v / per;
+    ok = true;
+    if (ids != nullptr) {
+      grp = ids[grp];
+      ok = grp >= 0 && grp < id_limit;
+    }
+    return grp * stride + off + v % per;
+  };
   for (int64_t v0 = warp; v0 < nvec; v0 += 2 * nwarps) {
     const int64_t v1 = v0 + nwarps;
-    const int64_t r0 = (v0 / per) * stride + off + v0 % per;
-    const int64_t r1 = (v1 / per) * stride + off + v1 % per;
-    typename R::type x0 = R::load(src + r0 * kD, lane);
-    typename R::type x1;
+    bool ok0, ok1 = false;
+    const int64_t r0 = row_of(v0, ok0);
     const bool has1 = v1 < nvec;
-    if (has1) x1 = R::load(src + r1 * kD, lane);
-    float a[4];
-    R::decode(x0, a);
-    dst[r0 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(a, t, lane));
-    if (has1) {
+    const int64_t r1 = has1 ? row_of(v1, ok1) : 0;
+    typename R::type x0, x1;
+    if (ok0) x0 = R::load(src + r0 * kD, lane);
+    if (ok1) x1 = R::load(src + r1 * kD, lane);
+    if (ok0) {
+      float a[4];
+      R::decode(x0, a);
+      dst[r0 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(a, t, lane));
+    }
+    if (ok1) {
       float b[4];
       R::decode(x1, b);
       dst[r1 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(b, t, lane));
@@ -49,16 +65,17 @@ static int encode_grid(int64_t nvec, int sms) {
 
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const int32_t* ids, int64_t id_limit) {
   if (nvec <= 0) return cudaSuccess;
   const int sms = current_device_sms(nullptr);
   const int grid = encode_grid(nvec, sms > 0 ? sms : 148);
   if (dt == ADAMAS_BF16) {
     encode_rows_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, t);
+        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, t, ids, id_limit);
   } else {
     encode_rows_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(src), dst,
-                                                         nvec, per, stride, off, t);
+                                                         nvec, per, stride, off, t, ids,
+                                                         id_limit);
   }
   return cudaGetLastError();
 }

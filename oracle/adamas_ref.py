@@ -285,3 +285,42 @@ def decode_step_varlen(q: np.ndarray, K: np.ndarray, V: np.ndarray, seq_lens, k:
         idx[b, :, :ib.shape[-1]] = ib[0]
         out[b] = ob[0]
     return idx, out
+
+
+# ------------------------------------------ dynamic (absmax) bucket thresholds
+def absmax_thresholds(x: np.ndarray, ratio: float = 0.5) -> np.ndarray:
+    """Per-vector threshold t_v = ratio * max_i |y_i| of the rotated vector y = H x / sqrt(d).
+
+    Blog "ADAMAS：稀疏注意力优化技术解析与应用实践", section 2.2: the bucket
+    thresholds are -0.5 absmax, 0, +0.5 absmax of the values being bucketed, and
+    groups of 128 dimensions beat one global absmax.  Reading: one group per head
+    vector (d = 128), the absmax taken after the Hadamard rotation (the values that
+    are bucketed), ratio 0.5 by default; float64, not rounded.
+    """
+    y = hadamard_rotate(x)
+    return float(ratio) * np.abs(y).max(axis=-1)
+
+
+def bucketize_per_vector(y: np.ndarray, t: np.ndarray) -> np.ndarray:
+    """bucketize with one threshold per vector (t has y's shape minus the last axis)."""
+    y = np.asarray(y, dtype=np.float64)
+    tt = np.asarray(t, dtype=np.float64)[..., None]
+    codes = np.full(y.shape, 3, dtype=np.uint8)
+    codes[y < tt] = 2
+    codes[y < 0.0] = 1
+    codes[y < -tt] = 0
+    return codes
+
+
+def encode_absmax(x: np.ndarray, ratio: float = 0.5) -> np.ndarray:
+    """Packed codes with per-vector absmax thresholds (see absmax_thresholds)."""
+    return pack_codes(bucketize_per_vector(hadamard_rotate(x), absmax_thresholds(x, ratio)))
+
+
+def decode_step_absmax(q: np.ndarray, K: np.ndarray, V: np.ndarray, k: int,
+                       ratio: float = 0.5, shared: bool = False):
+    """decode_step (or decode_step_shared) with every key and query encoded under its
+    own absmax threshold instead of one fixed t."""
+    step = decode_step_shared if shared else decode_step
+    return step(q, K, V, k, 0.0, key_codes=encode_absmax(K, ratio),
+                query_codes=encode_absmax(q, ratio))

@@ -20,6 +20,9 @@ What pins what:
 * Shared selection: G = 1 reduction, pure-Python brute force, identical heads.
 * Per-sequence lengths: pure-Python brute force (empty, short and long sequences,
   -1 padding), invariance to cache slots past a length, full-length reduction.
+* Absmax thresholds: hand-worked cases (tests/golden/absmax_cases.txt), reduction to
+  the fixed-threshold bucketize, the extreme coordinate's end bucket, per-vector
+  scale invariance, and a brute-force decode over the absmax codes.
 """
 from __future__ import annotations
 
@@ -387,6 +390,87 @@ def check_varlen_uniform_is_decode_step():
     assert np.array_equal(i1, i2) and np.array_equal(o1, o2)
 
 
+# ------------------------------------------- dynamic (absmax) thresholds
+def check_absmax_golden():
+    """Hand-worked per-vector thresholds (tests/golden/absmax_cases.txt)."""
+    cases = {}
+    for case, ratio, idx, y, want in _golden("absmax_cases.txt"):
+        cases.setdefault(int(case), (float(ratio), {}))[1][int(idx)] = (float(y), int(want))
+    for case, (ratio, entries) in cases.items():
+        y = np.zeros(128)
+        for i, (v, _) in entries.items():
+            y[i] = v
+        x = ref.hadamard_rotate(y)               # H / sqrt(d) is its own inverse
+        t = ref.absmax_thresholds(x, ratio)
+        assert abs(t - ratio * np.abs(y).max()) <= 1e-12 * np.abs(y).max(), (case, t)
+        codes = ref.unpack_codes(ref.encode_absmax(x, ratio))
+        for i, (_, want) in entries.items():
+            assert codes[i] == want, (case, i, codes[i], want)
+
+
+def check_bucket_per_vector_golden():
+    """The per-vector bucketize on the hand-worked threshold cases
+    (tests/golden/bucket_cases.txt, values on and beside each threshold), each case a
+    one-coordinate vector with its own t."""
+    rows = _golden("bucket_cases.txt")
+    t = np.array([float(r[0]) for r in rows])
+    y = np.array([[float(r[1])] for r in rows])
+    want = np.array([int(r[2]) for r in rows])
+    assert np.array_equal(ref.bucketize_per_vector(y, t)[:, 0], want)
+
+
+def check_absmax_reduces_to_fixed():
+    """With each vector's threshold handed to the fixed-threshold bucketize, the
+    per-vector rule gives the same codes."""
+    rng = np.random.default_rng(59)
+    x = rng.standard_normal((6, 128)) * rng.uniform(0.1, 10, (6, 1))
+    y = ref.hadamard_rotate(x)
+    t = np.float32(ref.absmax_thresholds(x, 0.5)).astype(np.float64)
+    per_vec = ref.bucketize_per_vector(y, t)
+    for v in range(6):
+        assert np.array_equal(per_vec[v], ref.bucketize(y[v], t[v]))
+
+
+def check_absmax_extreme_coordinate():
+    """ratio <= 1: the coordinate of largest magnitude always lands in an end bucket."""
+    rng = np.random.default_rng(61)
+    x = rng.standard_normal((50, 128))
+    y = ref.hadamard_rotate(x)
+    codes = ref.unpack_codes(ref.encode_absmax(x, 0.7))
+    j = np.abs(y).argmax(-1)
+    for v in range(50):
+        assert codes[v, j[v]] == (3 if y[v, j[v]] > 0 else 0)
+
+
+def check_absmax_per_vector_scale_invariance():
+    """Scaling one vector by a power of two leaves its codes and every other vector's
+    codes unchanged (the threshold is per vector, not global)."""
+    rng = np.random.default_rng(67)
+    x = rng.standard_normal((8, 128))
+    scales = 2.0 ** np.arange(-4, 4)[:, None]
+    a = ref.encode_absmax(x, 0.5)
+    b = ref.encode_absmax(x * scales, 0.5)
+    assert np.array_equal(a, b)
+
+
+def check_decode_absmax_uses_both_codes():
+    """decode_step_absmax = decode_step over the absmax codes of keys and queries."""
+    rng = np.random.default_rng(71)
+    q = rng.standard_normal((1, 4, 128))
+    K = rng.standard_normal((1, 2, 80, 128)) * rng.uniform(0.2, 5, (1, 2, 80, 1))
+    V = rng.standard_normal((1, 2, 80, 128))
+    i1, o1 = ref.decode_step_absmax(q, K, V, 11, 0.5)
+    cq = ref.unpack_codes(ref.encode_absmax(q, 0.5))
+    ck = ref.unpack_codes(ref.encode_absmax(K, 0.5))
+    for h in range(4):
+        d = [int(np.abs(cq[0, h].astype(int) - ck[0, h // 2, j].astype(int)).sum())
+             for j in range(80)]
+        want = _brute_select(d, 11)
+        assert list(i1[0, h]) == want
+        assert np.allclose(o1[0, h], _dense(q[0, h], K[0, h // 2, want], V[0, h // 2, want]),
+                           atol=1e-12)
+
+
 ALL_CHECKS = [
     check_hadamard_matches_scipy, check_hadamard_orthogonal,
     check_rotate_involution_and_dot, check_rotate_closed_forms, check_bucket_golden,
@@ -396,4 +480,6 @@ ALL_CHECKS = [
     check_gqa_and_planted, check_planted_recall_single_head,
     check_shared_g1_is_per_head, check_shared_bruteforce, check_shared_identical_heads,
     check_varlen_bruteforce, check_varlen_ignores_tail, check_varlen_uniform_is_decode_step,
+    check_absmax_golden, check_bucket_per_vector_golden, check_absmax_reduces_to_fixed, check_absmax_extreme_coordinate,
+    check_absmax_per_vector_scale_invariance, check_decode_absmax_uses_both_codes,
 ]

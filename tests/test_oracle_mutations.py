@@ -12,7 +12,8 @@ from pins import ALL_CHECKS
 _orig = {name: getattr(ref, name) for name in (
     "sylvester_hadamard", "hadamard_rotate", "bucketize", "pack_codes", "unpack_codes",
     "manhattan", "select_topk", "sparse_attention", "decode_step", "decode_step_shared",
-    "decode_step_varlen")}
+    "decode_step_varlen", "absmax_thresholds", "bucketize_per_vector", "encode_absmax",
+    "decode_step_absmax")}
 
 
 def _h_or(n=128):                      # popcount(i | j) instead of i & j
@@ -135,6 +136,38 @@ def _varlen_off_by_one(q, K, V, seq_lens, k, t, key_codes=None, query_codes=None
     return _orig["decode_step_varlen"](q, K, V, lens, k, t, shared=shared)
 
 
+def _absmax_unrotated(x, ratio=0.5):
+    # absmax of the raw vector instead of the rotated one
+    return float(ratio) * np.abs(np.asarray(x, np.float64)).max(axis=-1)
+
+
+def _absmax_global(x, ratio=0.5):
+    # one absmax over the whole tensor instead of per vector
+    y = _orig["hadamard_rotate"](x)
+    return np.full(y.shape[:-1], float(ratio) * np.abs(y).max())
+
+
+def _absmax_inverse_ratio(x, ratio=0.5):
+    return _orig["absmax_thresholds"](x, 1.0 / ratio)
+
+
+def _per_vector_le(y, t):
+    # "<=" instead of "<"
+    y = np.asarray(y, np.float64)
+    tt = np.asarray(t, np.float64)[..., None]
+    c = np.full(y.shape, 3, np.uint8)
+    c[y <= tt] = 2
+    c[y <= 0] = 1
+    c[y <= -tt] = 0
+    return c
+
+
+def _decode_absmax_fixed_query(q, K, V, k, ratio=0.5, shared=False):
+    # queries encoded with a fixed t = ratio instead of their own absmax threshold
+    step = _orig["decode_step_shared"] if shared else _orig["decode_step"]
+    return step(q, K, V, k, ratio, key_codes=_orig["encode_absmax"](K, ratio))
+
+
 MUTATIONS = {
     "hadamard_or": ("sylvester_hadamard", _h_or),
     "rotate_unscaled": ("hadamard_rotate", _rotate_unscaled),
@@ -153,6 +186,11 @@ MUTATIONS = {
     "varlen_full_cache": ("decode_step_varlen", _varlen_full_cache),
     "varlen_zero_pad": ("decode_step_varlen", _varlen_zero_pad),
     "varlen_off_by_one": ("decode_step_varlen", _varlen_off_by_one),
+    "absmax_unrotated": ("absmax_thresholds", _absmax_unrotated),
+    "absmax_global": ("absmax_thresholds", _absmax_global),
+    "absmax_inverse_ratio": ("absmax_thresholds", _absmax_inverse_ratio),
+    "absmax_bucket_le": ("bucketize_per_vector", _per_vector_le),
+    "absmax_fixed_query": ("decode_step_absmax", _decode_absmax_fixed_query),
 }
 
 

@@ -1,7 +1,8 @@
 """Benchmark of the Adamas decode step on B200: µs per step and effective HBM GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--budget 128]
-                    [--shared] [--paged PAGE] [--impl ours|reference]
+                    [--shared] [--paged PAGE] [--thresholds fixed|absmax]
+                    [--impl ours|reference]
 
 Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32 query / 8 kv heads,
 d = 128, context 32768, bf16 K/V with 4 outlier channels, budget 128.  A "step" is
@@ -168,11 +169,18 @@ def run_ours(args, rank, world, local):
     L = w.L
     t = w.t
     # one "set" = everything one decode step touches: per layer (q, K, V, codes)
+    absmax = args.thresholds == "absmax"
+    ratio = 0.5
+    if absmax and (args.paged or w.append):
+        raise SystemExit("--thresholds absmax is measured on contiguous caches without append")
     layer_sets = []
     for layer in range(w.layers):
         inp = generate(w, dev, layer=layer)
         codes = torch.empty(inp.k_cache.shape[:-1] + (32,), dtype=torch.uint8, device=dev)
-        ad.encode_keys(inp.k_cache, codes, 0, L, t)
+        if absmax:
+            ad.encode_keys_absmax(inp.k_cache, codes, 0, L, ratio)
+        else:
+            ad.encode_keys(inp.k_cache, codes, 0, L, t)
         layer_sets.append((inp.q, inp.k_cache, inp.v_cache, codes))
         del inp
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -222,6 +230,10 @@ def run_ours(args, rank, world, local):
                 continue
             if append:
                 ad.encode_keys(kc, cd, L - append, append, t, stream=s)
+            if absmax:
+                ad.decode_step_absmax(qq, kc, vc, cd, L, k, ratio, ws, shared=shared, out=o,
+                                      stream=s)
+                continue
             decode(qq, kc, vc, cd, L, k, t, ws, out=o, stream=s)
 
     # eager warm-up (also loads the kernels and sets their attributes)
@@ -301,16 +313,20 @@ def run_ours(args, rank, world, local):
     # per layer one C call: pinned q in, fused decode, fp32 out back to pinned host;
     # the calls are bound to their buffers once, as a serving loop would
     calls = None
-    if pc is None:
+    if pc is None and not absmax:
         calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws,
                                         outs[li], out_host[li], stream=stream, shared=shared)
                   for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
 
     def e2e_step(i):
         if calls is None:
-            # paged caches: the host copies around the public paged entry point
+            # paged caches / absmax thresholds: the host copies around the public call
             q_dev.copy_(q_host, non_blocking=True)
             for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
+                if pc is None:
+                    ad.decode_step_absmax(q_dev[li], kc, vc, cd, L, k, ratio, ws, shared=shared,
+                                          out=outs[li], stream=stream)
+                    continue
                 if append:
                     ad.encode_pages(kc, cd, t, page_ids=app_ids, stream=stream)
                 ad.decode_step_paged(q_dev[li], kc, vc, cd, bt, lens, L, k, t, ws, shared=shared,
@@ -355,16 +371,18 @@ def oracle_inputs(w, seed_device="cpu"):
     return inp.t, q, K, V, oracle
 
 
-def cpu_baseline(w, k, budget_s=12.0, shared=False):
+def cpu_baseline(w, k, budget_s=12.0, shared=False, absmax=False):
     """The oracle's full decode step (all heads) on the host, repeated for about
     budget_s seconds: effective GB/s over the same algorithmic bytes."""
     t, q, K, V, oracle = oracle_inputs(w)
-    kc = oracle.encode(K, t)        # key codes are cache state, built before timing
+    # key codes are cache state, built before timing; the query encode is timed
+    kc = oracle.encode_absmax(K, 0.5) if absmax else oracle.encode(K, t)
     fn = oracle.decode_step_shared if shared else oracle.decode_step
     n = 0
     t0 = time.perf_counter()
     while True:
-        fn(q, K, V, k, t, key_codes=kc)
+        qc = oracle.encode_absmax(q, 0.5) if absmax else None
+        fn(q, K, V, k, t, key_codes=kc, query_codes=qc)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 50:
@@ -441,6 +459,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shared", action="store_true",
                     help="shared GQA selection (one top-k per kv head)")
+    ap.add_argument("--thresholds", default="fixed", choices=["fixed", "absmax"],
+                    help="bucket thresholds: one fixed t, or per-vector 0.5 x absmax")
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE",
                     help="hold the caches in a pool of PAGE-token pages (block tables)")
     args = ap.parse_args()
@@ -466,7 +486,8 @@ def main():
     value = aggregate_gbs(r["step_bytes"], per_step_s, world)
     e2e_step_s = r["ms_e2e"] / 1e3 / r["K2"]
     key = (f"config{args.config}_k{k}" + ("_shared" if args.shared else "")
-           + (f"_paged{args.paged}" if args.paged else ""))
+           + (f"_paged{args.paged}" if args.paged else "")
+           + ("_absmax" if args.thresholds == "absmax" else ""))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -486,6 +507,8 @@ def main():
                    "k": k, "algorithmic_bytes_per_step": r["step_bytes"],
                    "selection": "shared per kv head" if args.shared else "per query head",
                    "cache": f"paged, {args.paged}-token pages" if args.paged else "contiguous",
+                   "thresholds": ("per-vector 0.5 x absmax" if args.thresholds == "absmax"
+                                  else "fixed t"),
                    "replicas": r["R"], "l2": "rotated replicas, working set >= 2x L2",
                    "layers": w.layers, "append_tokens": w.append,
                    "graph": r["use_graph"], "ctas": r["plan"]["ctas"],
@@ -502,7 +525,8 @@ def main():
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, k, shared=args.shared)
+        line["cpu_baseline"] = cpu_baseline(w, k, shared=args.shared,
+                                            absmax=args.thresholds == "absmax")
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -247,6 +247,36 @@ adamas_status adamas_encode_pages(const void* k_pages, adamas_dtype dt, int Hkv,
                                   int64_t n_ids, float t, uint8_t* code_pages,
                                   cudaStream_t stream);
 
+/*
+ * Dynamic (per-vector) bucket thresholds: blog "ADAMAS：稀疏注意力优化技术解析与应用实践",
+ * section 2.2, sets the thresholds at -0.5 absmax, 0, +0.5 absmax of the values being
+ * bucketed, with groups of 128 dimensions.  Here every key and query vector (one
+ * 128-dimension group) gets t_v = ratio * max_i |y_i| of its own rotated values y;
+ * 0 < ratio <= 1 (the blog's 0.5); other values return ADAMAS_ERR_INVALID_ARG.
+ * Layouts and errors are those of the fixed-threshold encoders.
+ */
+adamas_status adamas_encode_keys_absmax(const void* k_cache, adamas_dtype dt, int B, int Hkv,
+                                        int d, int64_t Lmax, int64_t pos0, int64_t n_new,
+                                        float ratio, uint8_t* codes, cudaStream_t stream);
+adamas_status adamas_encode_queries_absmax(const void* q, adamas_dtype dt, int B, int Hq, int d,
+                                           float ratio, uint8_t* qcodes, cudaStream_t stream);
+adamas_status adamas_encode_pages_absmax(const void* k_pages, adamas_dtype dt, int Hkv, int d,
+                                         int page_size, int64_t num_pages,
+                                         const int32_t* page_ids, int64_t n_ids, float ratio,
+                                         uint8_t* code_pages, cudaStream_t stream);
+
+/*
+ * adamas_decode_step (shared = 0) or adamas_decode_step_shared (shared = 1) with the
+ * fused query encode using per-vector absmax thresholds; `codes` must hold keys
+ * encoded by adamas_encode_keys_absmax with the same ratio.
+ */
+adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, int64_t L, int k,
+                                        float ratio, int shared, void* workspace,
+                                        size_t ws_bytes, int32_t* idx_out, float* out,
+                                        cudaStream_t stream);
+
 /* Workspace of adamas_sparse_attention, in bytes (zero-filled once, self-cleaning). */
 size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff);
 

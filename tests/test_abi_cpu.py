@@ -198,3 +198,22 @@ def test_paging_helper_layout():
             assert torch.equal(pool[page, :, p % 16], x[b, :, p])
     spare = set(range(pc.num_pages)) - set(used)
     assert all((pool[s] == -1).all() for s in spare)
+
+
+def test_absmax_entry_points_reject():
+    ek = ad.lib().adamas_encode_keys_absmax
+    for ratio in (0.0, -0.5, 1.5, math.nan, math.inf):
+        assert ek(A, BF16, 1, 8, 128, 100, 0, 10, ratio, A, None) == ERR_INVALID_ARG, ratio
+    assert ek(A, BF16, 1, 8, 96, 100, 0, 10, 0.5, A, None) == ERR_UNSUPPORTED
+    eq = ad.lib().adamas_encode_queries_absmax
+    assert eq(A, BF16, 1, 32, 128, 0.0, A, None) == ERR_INVALID_ARG
+    assert eq(A, BF16, 1, 32, 128, 0.5, None, None) == ERR_INVALID_ARG
+    ep = ad.lib().adamas_encode_pages_absmax
+    assert ep(A, BF16, 8, 128, 16, 100, None, 0, 2.0, A, None) == ERR_INVALID_ARG
+    d = ad.lib().adamas_decode_step_absmax
+    ok = [A, A, A, A, BF16, 1, 32, 8, 128, 4096, 4096, 128, 0.5, 0, A, 1 << 30, None, A, None]
+    for i, bad in [(12, 0.0), (12, 1.01), (13, 3), (0, None), (14, A + 16), (15, 16)]:
+        args = list(ok); args[i] = bad
+        assert d(*args) == ERR_INVALID_ARG, (i, bad)
+    args = list(ok); args[6] = 24
+    assert d(*args) == ERR_UNSUPPORTED

@@ -70,6 +70,14 @@ _SIGNATURES = {
                                         _c_p, _c_i64, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p]),
     "adamas_encode_pages": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_p, _c_i64, _c_f,
                                    _c_p, _c_p]),
+    "adamas_encode_keys_absmax": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i64,
+                                         _c_f, _c_p, _c_p]),
+    "adamas_encode_queries_absmax": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p]),
+    "adamas_encode_pages_absmax": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_p, _c_i64,
+                                          _c_f, _c_p, _c_p]),
+    "adamas_decode_step_absmax": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                         _c_i64, _c_i64, _c_i, _c_f, _c_i, _c_p, _c_sz, _c_p,
+                                         _c_p, _c_p]),
     "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "adamas_sparse_attention": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i, _c_i,
                                        _c_i64, _c_i, _c_p, _c_sz, _c_p, _c_p]),
@@ -396,6 +404,60 @@ def encode_pages(k_pages, code_pages, t: float, page_ids=None, stream=None):
                                      P, ids, n, float(t), _dev(code_pages, "code_pages"),
                                      _stream(stream)), "adamas_encode_pages")
     return code_pages
+
+
+# --------------------------------------------- per-vector absmax thresholds
+def encode_keys_absmax(k_cache: torch.Tensor, codes: torch.Tensor, pos0: int, n_new: int,
+                       ratio: float = 0.5, stream=None):
+    """encode_keys with each key's threshold ratio * max |H k / sqrt(d)|."""
+    B, Hkv, Lmax, d = k_cache.shape
+    if codes.dtype != torch.uint8 or tuple(codes.shape) != (B, Hkv, Lmax, d // 4):
+        raise ValueError("codes must be uint8 [B, Hkv, Lmax, d/4]")
+    _check(lib().adamas_encode_keys_absmax(_dev(k_cache, "k_cache"), _dtype_code(k_cache), B, Hkv,
+                                           d, Lmax, pos0, n_new, float(ratio),
+                                           _dev(codes, "codes"), _stream(stream)),
+           "adamas_encode_keys_absmax")
+    return codes
+
+
+def encode_queries_absmax(q: torch.Tensor, ratio: float = 0.5, qcodes=None, stream=None):
+    B, Hq, d = q.shape
+    if qcodes is None:
+        qcodes = torch.empty((B, Hq, d // 4), dtype=torch.uint8, device=q.device)
+    _check(lib().adamas_encode_queries_absmax(_dev(q, "q"), _dtype_code(q), B, Hq, d,
+                                              float(ratio), _dev(qcodes, "qcodes"),
+                                              _stream(stream)), "adamas_encode_queries_absmax")
+    return qcodes
+
+
+def encode_pages_absmax(k_pages, code_pages, ratio: float = 0.5, page_ids=None, stream=None):
+    P, Hkv, page, d = k_pages.shape
+    if code_pages.dtype != torch.uint8 or tuple(code_pages.shape) != (P, Hkv, page, d // 4):
+        raise ValueError("code_pages must be uint8 [P, Hkv, page, d/4]")
+    ids = None if page_ids is None else _i32(page_ids, "page_ids")
+    n = 0 if page_ids is None else page_ids.numel()
+    _check(lib().adamas_encode_pages_absmax(_dev(k_pages, "k_pages"), _dtype_code(k_pages), Hkv, d,
+                                            page, P, ids, n, float(ratio),
+                                            _dev(code_pages, "code_pages"), _stream(stream)),
+           "adamas_encode_pages_absmax")
+    return code_pages
+
+
+def decode_step_absmax(q, k_cache, v_cache, codes, L: int, k: int, ratio: float, ws,
+                       shared: bool = False, idx_out=None, out=None, stream=None):
+    """Decode step whose fused query encode uses per-vector absmax thresholds (codes
+    from encode_keys_absmax with the same ratio)."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
+    _check(lib().adamas_decode_step_absmax(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(codes, "codes"),
+        _dtype_code(k_cache), B, Hq, Hkv, d, Lmax, L, k, float(ratio), int(bool(shared)),
+        _dev(ws, "workspace"), ws.numel(), idx_ptr, _dev(out, "out"), _stream(stream)),
+        "adamas_decode_step_absmax")
+    return out
 
 
 def sparse_attention_workspace(B: int, Hq: int, k_eff: int, device="cuda", stream=None):

@@ -46,6 +46,53 @@ CacheLayout contiguous(int64_t Lmax) {
   return c;
 }
 
+// Encoders with a fixed threshold t (ratio == 0) or per-vector absmax thresholds
+// (0 < ratio <= 1; t unused).
+bool good_threshold(float t, float ratio) {
+  if (ratio == 0.0f) return good_t(t);
+  return std::isfinite(ratio) && ratio > 0.0f && ratio <= 1.0f;
+}
+
+adamas_status encode_keys_common(const void* k_cache, adamas_dtype dt, int B, int Hkv, int d,
+                                 int64_t Lmax, int64_t pos0, int64_t n_new, float t, float ratio,
+                                 uint8_t* codes, cudaStream_t stream) {
+  if (!k_cache || !codes || !good_dtype(dt) || !good_threshold(t, ratio))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || Lmax <= 0 || pos0 < 0 || n_new <= 0 || pos0 + n_new > Lmax)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!aligned(k_cache, 16) || !aligned(codes, 16)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_encode_rows(k_cache, dt, codes, int64_t(B) * Hkv * n_new, n_new, Lmax,
+                                      pos0, t, stream, nullptr, 0, ratio));
+}
+
+adamas_status encode_queries_common(const void* q, adamas_dtype dt, int B, int Hq, int d,
+                                    float t, float ratio, uint8_t* qcodes, cudaStream_t stream) {
+  if (!q || !qcodes || !good_dtype(dt) || !good_threshold(t, ratio) || B <= 0 || Hq <= 0)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(qcodes, 16)) return ADAMAS_ERR_INVALID_ARG;
+  const int64_t n = int64_t(B) * Hq;
+  return from_cuda(launch_encode_rows(q, dt, qcodes, n, n, 0, 0, t, stream, nullptr, 0, ratio));
+}
+
+adamas_status encode_pages_common(const void* k_pages, adamas_dtype dt, int Hkv, int d,
+                                  int page_size, int64_t num_pages, const int32_t* page_ids,
+                                  int64_t n_ids, float t, float ratio, uint8_t* code_pages,
+                                  cudaStream_t stream) {
+  if (!k_pages || !code_pages || !good_dtype(dt) || !good_threshold(t, ratio))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
+  if (Hkv <= 0 || page_size < 1 || num_pages < 1 || num_pages > INT32_MAX)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (page_ids && (n_ids < 0 || !aligned(page_ids, 4))) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(k_pages, 16) || !aligned(code_pages, 16)) return ADAMAS_ERR_INVALID_ARG;
+  const int64_t per = int64_t(Hkv) * page_size;           // rows per page
+  const int64_t groups = page_ids ? n_ids : num_pages;
+  return from_cuda(launch_encode_rows(k_pages, dt, code_pages, groups * per, per, per, 0, t,
+                                      stream, page_ids, num_pages, ratio));
+}
+
 // Device address of a page-locked, device-mapped host buffer; nullptr for any
 // other memory (pageable host memory, device memory, unknown pointers).
 template <typename P>
@@ -89,26 +136,72 @@ const char* adamas_status_string(adamas_status s) {
 
 int adamas_abi_version(void) { return 1; }
 
+
+
 adamas_status adamas_encode_keys(const void* k_cache, adamas_dtype dt, int B, int Hkv, int d,
                                  int64_t Lmax, int64_t pos0, int64_t n_new, float t,
                                  uint8_t* codes, cudaStream_t stream) {
-  if (!k_cache || !codes || !good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
-  if (B <= 0 || Hkv <= 0 || Lmax <= 0 || pos0 < 0 || n_new <= 0 || pos0 + n_new > Lmax)
-    return ADAMAS_ERR_INVALID_ARG;
-  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
-  if (!aligned(k_cache, 16) || !aligned(codes, 16)) return ADAMAS_ERR_INVALID_ARG;
-  return from_cuda(launch_encode_rows(k_cache, dt, codes, int64_t(B) * Hkv * n_new, n_new, Lmax,
-                                      pos0, t, stream));
+  return encode_keys_common(k_cache, dt, B, Hkv, d, Lmax, pos0, n_new, t, 0.0f, codes, stream);
+}
+
+adamas_status adamas_encode_keys_absmax(const void* k_cache, adamas_dtype dt, int B, int Hkv,
+                                        int d, int64_t Lmax, int64_t pos0, int64_t n_new,
+                                        float ratio, uint8_t* codes, cudaStream_t stream) {
+  if (!(ratio > 0.0f)) return ADAMAS_ERR_INVALID_ARG;
+  return encode_keys_common(k_cache, dt, B, Hkv, d, Lmax, pos0, n_new, 0.0f, ratio, codes,
+                            stream);
 }
 
 adamas_status adamas_encode_queries(const void* q, adamas_dtype dt, int B, int Hq, int d,
                                     float t, uint8_t* qcodes, cudaStream_t stream) {
-  if (!q || !qcodes || !good_dtype(dt) || !good_t(t) || B <= 0 || Hq <= 0)
+  return encode_queries_common(q, dt, B, Hq, d, t, 0.0f, qcodes, stream);
+}
+
+adamas_status adamas_encode_queries_absmax(const void* q, adamas_dtype dt, int B, int Hq, int d,
+                                           float ratio, uint8_t* qcodes, cudaStream_t stream) {
+  if (!(ratio > 0.0f)) return ADAMAS_ERR_INVALID_ARG;
+  return encode_queries_common(q, dt, B, Hq, d, 0.0f, ratio, qcodes, stream);
+}
+
+adamas_status adamas_encode_pages(const void* k_pages, adamas_dtype dt, int Hkv, int d,
+                                  int page_size, int64_t num_pages, const int32_t* page_ids,
+                                  int64_t n_ids, float t, uint8_t* code_pages,
+                                  cudaStream_t stream) {
+  return encode_pages_common(k_pages, dt, Hkv, d, page_size, num_pages, page_ids, n_ids, t, 0.0f,
+                             code_pages, stream);
+}
+
+adamas_status adamas_encode_pages_absmax(const void* k_pages, adamas_dtype dt, int Hkv, int d,
+                                         int page_size, int64_t num_pages,
+                                         const int32_t* page_ids, int64_t n_ids, float ratio,
+                                         uint8_t* code_pages, cudaStream_t stream) {
+  if (!(ratio > 0.0f)) return ADAMAS_ERR_INVALID_ARG;
+  return encode_pages_common(k_pages, dt, Hkv, d, page_size, num_pages, page_ids, n_ids, 0.0f,
+                             ratio, code_pages, stream);
+}
+
+adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, int64_t L, int k,
+                                        float ratio, int shared, void* workspace,
+                                        size_t ws_bytes, int32_t* idx_out, float* out,
+                                        cudaStream_t stream) {
+  if (!(ratio > 0.0f) || !good_threshold(0.0f, ratio) || (shared != 0 && shared != 1))
     return ADAMAS_ERR_INVALID_ARG;
-  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(qcodes, 16)) return ADAMAS_ERR_INVALID_ARG;
-  const int64_t n = int64_t(B) * Hq;
-  return from_cuda(launch_encode_rows(q, dt, qcodes, n, n, 0, 0, t, stream));
+  if (!q || !k_cache || !v_cache || !codes || !workspace || !out) return ADAMAS_ERR_INVALID_ARG;
+  if (!good_dtype(dt)) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(codes, 16) ||
+      !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
+                                 contiguous(Lmax), L, k, 0.0f, workspace, idx_out, out,
+                                 shared != 0, p, stream, ratio));
 }
 
 size_t adamas_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k) {
@@ -391,21 +484,6 @@ adamas_status adamas_select_topk_paged(const uint8_t* qcodes, const uint8_t* cod
                        nullptr, stream);
 }
 
-adamas_status adamas_encode_pages(const void* k_pages, adamas_dtype dt, int Hkv, int d,
-                                  int page_size, int64_t num_pages, const int32_t* page_ids,
-                                  int64_t n_ids, float t, uint8_t* code_pages,
-                                  cudaStream_t stream) {
-  if (!k_pages || !code_pages || !good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
-  if (d != kD) return ADAMAS_ERR_UNSUPPORTED;
-  if (Hkv <= 0 || page_size < 1 || num_pages < 1 || num_pages > INT32_MAX)
-    return ADAMAS_ERR_INVALID_ARG;
-  if (page_ids && (n_ids < 0 || !aligned(page_ids, 4))) return ADAMAS_ERR_INVALID_ARG;
-  if (!aligned(k_pages, 16) || !aligned(code_pages, 16)) return ADAMAS_ERR_INVALID_ARG;
-  const int64_t per = int64_t(Hkv) * page_size;           // rows per page
-  const int64_t groups = page_ids ? n_ids : num_pages;
-  return from_cuda(launch_encode_rows(k_pages, dt, code_pages, groups * per, per, per, 0, t,
-                                      stream, page_ids, num_pages));
-}
 
 adamas_status adamas_select_topk_shared(const uint8_t* qcodes, const uint8_t* codes, int B,
                                         int Hq, int Hkv, int64_t Lmax, int64_t L, int k,

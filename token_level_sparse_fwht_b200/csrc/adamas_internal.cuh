@@ -208,8 +208,11 @@ template <> struct Raw4<__nv_bfloat16> {
 // (lane l: elements 4l..4l+3), natural (Sylvester) order, fp32.  Index bits 0-1
 // are butterflied inside the lane, bits 2-6 across lanes with xor-shuffles.
 // Returns the lane's byte of the packed code: 4 coordinates, 2 bits each,
-// coordinate 4l+r at bits 2r, code = [y >= -t] + [y >= 0] + [y >= t].
-__device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane) {
+// coordinate 4l+r at bits 2r, code = [y >= -t] + [y >= 0] + [y >= t].  With
+// ratio > 0 the threshold is the vector's own: t = ratio * max_i |y_i| (blog
+// "ADAMAS：稀疏注意力优化技术解析与应用实践", section 2.2, one 128-dimension group).
+__device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane,
+                                                   float ratio = 0.0f) {
   const float a0 = v[0] + v[1], a1 = v[0] - v[1];
   const float a2 = v[2] + v[3], a3 = v[2] - v[3];
   v[0] = a0 + a2; v[1] = a1 + a3; v[2] = a0 - a2; v[3] = a1 - a3;
@@ -223,11 +226,18 @@ __device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane
     }
   }
   const float inv_sqrt_d = 0.088388347648318440550f;   // 1 / sqrt(128)
+#pragma unroll
+  for (int r = 0; r < 4; ++r) v[r] *= inv_sqrt_d;
+  if (ratio > 0.0f) {
+    float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, s));
+    t = ratio * m;
+  }
   uint32_t byte = 0;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    const float y = v[r] * inv_sqrt_d;
-    v[r] = y;
+    const float y = v[r];
     const uint32_t c = (uint32_t)(y >= -t) + (uint32_t)(y >= 0.0f) + (uint32_t)(y >= t);
     byte |= c << (2 * r);
   }
@@ -506,11 +516,11 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
                           const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
                           int32_t* idx_out, float* out, bool shared, const Plan& p,
-                          cudaStream_t stream);
+                          cudaStream_t stream, float t_ratio = 0.0f);
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
                                cudaStream_t stream, const int32_t* ids = nullptr,
-                               int64_t id_limit = 0);
+                               int64_t id_limit = 0, float ratio = 0.0f);
 size_t attention_workspace_bytes(int B, int Hq, int k_eff);
 bool noalloc_fits(int B, int Hq);
 cudaError_t launch_sparse_attention_noalloc(const void* q, const void* k, const void* v,

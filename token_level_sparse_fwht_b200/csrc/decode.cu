@@ -64,6 +64,7 @@ struct DecodeArgs {
   int page_shift;            // log2(page size)
   int64_t num_pages;
   float t;
+  float t_ratio;             // > 0: each query's threshold is t_ratio * its rotated absmax
   float scale_log2;
   int32_t* idx_out;          // [B][rows][idx_stride] or nullptr (-1 past a unit's count)
   float* out;                // [B][Hq][128] or nullptr (select mode)
@@ -340,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       load4(static_cast<const T*>(a.q) + (int64_t(b) * a.Hq + h) * kD, lane, v);
       float* qrow = qf + g * kD + 4 * lane;
       qrow[0] = v[0]; qrow[1] = v[1]; qrow[2] = v[2]; qrow[3] = v[3];
-      qc[g * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(v, a.t, lane));
+      qc[g * kCodeBytes + lane] =
+          static_cast<uint8_t>(warp_fwht_code(v, a.t, lane, a.t_ratio));
     }
   }
   __syncthreads();
@@ -987,7 +989,7 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
                           const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
                           int32_t* idx_out, float* out, bool shared, const Plan& p,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, float t_ratio) {
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q; a.qcodes = qcodes; a.k = k; a.v = v; a.codes = codes;
@@ -1000,6 +1002,7 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.page_shift = lay.page_shift;
   a.num_pages = lay.num_pages;
   a.t = t;
+  a.t_ratio = t_ratio;
   a.scale_log2 = float(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   a.idx_out = idx_out; a.out = out;
   a.err = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + decode_workspace_error_offset());

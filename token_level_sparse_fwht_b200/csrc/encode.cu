@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ 
                                                           int64_t stride, int64_t off,
                                                           float t,
                                                           const int32_t* __restrict__ ids,
-                                                          int64_t id_limit) {
+                                                          int64_t id_limit, float ratio) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
@@ -46,12 +46,12 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ 
     if (ok0) {
       float a[4];
       R::decode(x0, a);
-      dst[r0 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(a, t, lane));
+      dst[r0 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(a, t, lane, ratio));
     }
     if (ok1) {
       float b[4];
       R::decode(x1, b);
-      dst[r1 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(b, t, lane));
+      dst[r1 * kCodeBytes + lane] = static_cast<uint8_t>(warp_fwht_code(b, t, lane, ratio));
     }
   }
 }
@@ -65,17 +65,19 @@ static int encode_grid(int64_t nvec, int sms) {
 
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
-                               cudaStream_t stream, const int32_t* ids, int64_t id_limit) {
+                               cudaStream_t stream, const int32_t* ids, int64_t id_limit,
+                               float ratio) {
   if (nvec <= 0) return cudaSuccess;
   const int sms = current_device_sms(nullptr);
   const int grid = encode_grid(nvec, sms > 0 ? sms : 148);
   if (dt == ADAMAS_BF16) {
     encode_rows_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, t, ids, id_limit);
+        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, t, ids, id_limit,
+        ratio);
   } else {
     encode_rows_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(src), dst,
                                                          nvec, per, stride, off, t, ids,
-                                                         id_limit);
+                                                         id_limit, ratio);
   }
   return cudaGetLastError();
 }

@@ -216,9 +216,39 @@ def run_ours(args, rank, world, local):
     out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
     plan = (ad.decode_plan_shared if shared else ad.decode_plan)(w.B, w.Hq, w.Hkv, L, k)
-    launches_per_step = w.layers * (2 if append else 1)
+    launches_per_step = w.layers * (2 if append else 1) * (1 if not args.cp else 3)
+
+    cpW = args.cp
+    if cpW:
+        # one rank of a context-parallel step over W GPUs, on one GPU: this rank holds
+        # the first L / W positions; both all-gathers are stood in for by a local copy
+        # of this rank's own tensor into the gathered buffer (the NCCL transfer itself
+        # is not timed)
+        if args.paged or absmax or append or w.layers > 1:
+            raise SystemExit("--cp is measured on one contiguous layer without append")
+        Ls = L // cpW
+        rows = w.Hkv if shared else w.Hq
+        hist_all = torch.empty((cpW,) + ad.cp_hist_shape(w.B, w.Hq, w.Hkv, shared),
+                               dtype=torch.int32, device=dev)
+        part_all = torch.empty((cpW, w.B, w.Hq, ad.PART_STRIDE), dtype=torch.float32,
+                               device=dev)
+        ws_cp = ad.cp_workspace(w.B, w.Hq, w.Hkv, Ls, k, shared, dev)
+        step_bytes = (w.B * w.Hkv * Ls * 32 + w.B * w.Hq * min(k, L) // cpW * 2 * 128
+                      * w.elem_bytes + w.B * w.Hq * 128 * (w.elem_bytes + 4))
 
     def step(i, s, q_override=None, out_t=None):
+        if cpW:
+            for (q, kc, vc, cd) in sets[i % R]:
+                qq = q if q_override is None else q_override
+                o = out if out_t is None else out_t
+                ad.cp_histograms(qq, cd, Ls, k, t, ws_cp, shared=shared, hist_out=hist_all[0],
+                                 stream=s)
+                hist_all[1:].copy_(hist_all[0].expand_as(hist_all[1:]))
+                ad.cp_attend(qq, kc, vc, cd, Ls, L, 0, k, t, hist_all, 0, ws_cp, shared=shared,
+                             partial_out=part_all[0], stream=s)
+                part_all[1:].copy_(part_all[0].expand_as(part_all[1:]))
+                ad.cp_combine(part_all, out=o, stream=s)
+            return
         for (q, kc, vc, cd) in sets[i % R]:
             qq = q if q_override is None else q_override
             o = out if out_t is None else out_t
@@ -313,12 +343,17 @@ def run_ours(args, rank, world, local):
     # per layer one C call: pinned q in, fused decode, fp32 out back to pinned host;
     # the calls are bound to their buffers once, as a serving loop would
     calls = None
-    if pc is None and not absmax:
+    if pc is None and not absmax and not cpW:
         calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws,
                                         outs[li], out_host[li], stream=stream, shared=shared)
                   for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
 
     def e2e_step(i):
+        if cpW:
+            q_dev.copy_(q_host, non_blocking=True)
+            step(i, stream, q_override=q_dev[0], out_t=outs[0])
+            out_host.copy_(outs, non_blocking=True)
+            return
         if calls is None:
             # paged caches / absmax thresholds: the host copies around the public call
             q_dev.copy_(q_host, non_blocking=True)
@@ -461,6 +496,8 @@ def main():
                     help="shared GQA selection (one top-k per kv head)")
     ap.add_argument("--thresholds", default="fixed", choices=["fixed", "absmax"],
                     help="bucket thresholds: one fixed t, or per-vector 0.5 x absmax")
+    ap.add_argument("--cp", type=int, default=0, metavar="W",
+                    help="time one rank of a W-way context-parallel step (its L/W slice)")
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE",
                     help="hold the caches in a pool of PAGE-token pages (block tables)")
     args = ap.parse_args()
@@ -487,7 +524,8 @@ def main():
     e2e_step_s = r["ms_e2e"] / 1e3 / r["K2"]
     key = (f"config{args.config}_k{k}" + ("_shared" if args.shared else "")
            + (f"_paged{args.paged}" if args.paged else "")
-           + ("_absmax" if args.thresholds == "absmax" else ""))
+           + ("_absmax" if args.thresholds == "absmax" else "")
+           + (f"_cp{args.cp}" if args.cp else ""))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -509,6 +547,8 @@ def main():
                    "cache": f"paged, {args.paged}-token pages" if args.paged else "contiguous",
                    "thresholds": ("per-vector 0.5 x absmax" if args.thresholds == "absmax"
                                   else "fixed t"),
+                   "context_parallel": (f"one rank of {args.cp}: L/{args.cp} slice, all-gathers "
+                                        "stood in for by local copies" if args.cp else None),
                    "replicas": r["R"], "l2": "rotated replicas, working set >= 2x L2",
                    "layers": w.layers, "append_tokens": w.append,
                    "graph": r["use_graph"], "ctas": r["plan"]["ctas"],

@@ -277,6 +277,54 @@ adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, cons
                                         size_t ws_bytes, int32_t* idx_out, float* out,
                                         cudaStream_t stream);
 
+/*
+ * Context-parallel decode (one GPU per contiguous slice of a long context).  The
+ * pages run one device; this split is the implementation's.  Rank r of `world`
+ * holds positions [pos_offset, pos_offset + L) of a context of L_total positions
+ * (lower ranks hold lower positions) in contiguous caches [B][Hkv][Lmax][d] and
+ * codes [B][Hkv][Lmax][d/4].  One step:
+ *   1. adamas_cp_histograms: per selection row (query head, or kv head if shared),
+ *      the cumulative histogram of Manhattan distances over the slice -> hist
+ *      [B][rows][bins] uint32 (count of distances <= bin), bins = 385 (per head) or
+ *      384 G + 1 (shared); adamas_cp_hist_elems gives B * rows * bins.
+ *   2. the caller all-gathers the histograms of all ranks, rank order:
+ *      hist_all [world][B][rows][bins].
+ *   3. adamas_cp_attend: the global top-k (the first min(k, L_total) positions by
+ *      (distance, global position)) restricted to this slice, attention over it,
+ *      and one softmax partial per query head -> partial [B][Hq][132] float
+ *      (m in the log2 domain, l, 0, 0, acc[128]; l = 0: nothing selected here).
+ *      idx_out (nullable, [B][rows][min(k, L_total)]) receives this rank's global
+ *      positions at their global slots; other slots are left untouched, so
+ *      -1-filled arrays of all ranks merge by elementwise max.
+ *   4. the caller all-gathers the partials: partials_all [world][B][Hq][132].
+ *   5. adamas_cp_combine: out [B][Hq][d] float, equal to adamas_decode_step (or
+ *      _shared) over the whole context.
+ * Steps 1 and 3 are launches of the fused decode kernel (q encoded inside, as in
+ * adamas_decode_step); step 3 reads back the distances step 1 computed (the codes
+ * are scanned once).  Errors as adamas_decode_step, plus ADAMAS_ERR_INVALID_ARG for
+ * pos_offset < 0, pos_offset + L > L_total, L_total > 2^31 - 1 or rank outside
+ * [0, world).
+ */
+size_t adamas_cp_hist_elems(int B, int Hq, int Hkv, int shared);
+/* Workspace of adamas_cp_histograms / adamas_cp_attend for this rank's L positions:
+ * the error word plus the distances and histograms each CTA keeps from step 1 to
+ * step 3 (zero-fill once with adamas_workspace_init; both steps must get the same
+ * workspace and sizes); 0 if the arguments are invalid. */
+size_t adamas_cp_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k, int shared);
+adamas_status adamas_cp_histograms(const void* q, const uint8_t* codes, adamas_dtype dt, int B,
+                                   int Hq, int Hkv, int d, int64_t Lmax, int64_t L, int k,
+                                   float t, int shared, void* workspace, size_t ws_bytes,
+                                   uint32_t* hist_out, cudaStream_t stream);
+adamas_status adamas_cp_attend(const void* q, const void* k_cache, const void* v_cache,
+                               const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
+                               int d, int64_t Lmax, int64_t L, int64_t L_total,
+                               int64_t pos_offset, int k, float t, int shared,
+                               const uint32_t* hist_all, int world, int rank, void* workspace,
+                               size_t ws_bytes, int32_t* idx_out, float* partial_out,
+                               cudaStream_t stream);
+adamas_status adamas_cp_combine(const float* partials_all, int world, int B, int Hq, float* out,
+                                cudaStream_t stream);
+
 /* Workspace of adamas_sparse_attention, in bytes (zero-filled once, self-cleaning). */
 size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff);
 

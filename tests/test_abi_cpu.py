@@ -217,3 +217,33 @@ def test_absmax_entry_points_reject():
         assert d(*args) == ERR_INVALID_ARG, (i, bad)
     args = list(ok); args[6] = 24
     assert d(*args) == ERR_UNSUPPORTED
+
+
+def test_context_parallel_entry_points_reject():
+    assert ad.lib().adamas_cp_hist_elems(2, 32, 8, 0) == 2 * 32 * 385
+    assert ad.lib().adamas_cp_hist_elems(2, 32, 8, 1) == 2 * 8 * (384 * 4 + 1)
+    assert ad.lib().adamas_cp_hist_elems(2, 24, 8, 0) == 0
+    h = ad.lib().adamas_cp_histograms
+    assert h(None, A, BF16, 1, 32, 8, 128, 100, 100, 10, 1.0, 0, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    assert h(A, A, BF16, 1, 32, 8, 128, 100, 100, 10, 1.0, 2, A, 1 << 30, A, None) == ERR_INVALID_ARG
+    at = ad.lib().adamas_cp_attend
+    ok = [A, A, A, A, BF16, 1, 32, 8, 128, 100, 100, 300, 100, 10, 1.0, 0, A, 2, 1, A, 1 << 30,
+          None, A, None]
+    for i, bad in [(12, -1), (11, 150), (11, 1 << 31), (16, None), (22, None), (17, 0), (18, 2),
+                   (18, -1)]:
+        args = list(ok); args[i] = bad
+        assert at(*args) == ERR_INVALID_ARG, (i, bad)
+    c = ad.lib().adamas_cp_combine
+    assert c(A, 0, 1, 32, A, None) == ERR_INVALID_ARG
+    assert c(None, 2, 1, 32, A, None) == ERR_INVALID_ARG
+
+
+def test_context_parallel_workspace_size():
+    # the error word plus, per CTA, its distances (u16 per key and selection head) and
+    # cumulative histograms
+    n = ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 128, 16384, 128, 0)
+    p = ad.decode_plan(1, 32, 8, 16384, 128)
+    per_cta = 4 * ((p["tokens_per_cta"] + 7) // 8 * 8) * 2 + 4 * 388 * 4
+    assert n == 256 + p["ctas"] * per_cta
+    assert ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 128, 16384, 128, 2) == 0
+    assert ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 64, 16384, 128, 0) == 0

@@ -78,6 +78,14 @@ _SIGNATURES = {
     "adamas_decode_step_absmax": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i,
                                          _c_i64, _c_i64, _c_i, _c_f, _c_i, _c_p, _c_sz, _c_p,
                                          _c_p, _c_p]),
+    "adamas_cp_hist_elems": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
+    "adamas_cp_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i64, _c_i, _c_i]),
+    "adamas_cp_histograms": (_c_i, [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_i64,
+                                    _c_i, _c_f, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "adamas_cp_attend": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i64,
+                                _c_i64, _c_i64, _c_i64, _c_i, _c_f, _c_i, _c_p, _c_i, _c_i,
+                                _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "adamas_cp_combine": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p]),
     "adamas_sparse_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i]),
     "adamas_sparse_attention": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_p, _c_i, _c_i, _c_i, _c_i,
                                        _c_i64, _c_i, _c_p, _c_sz, _c_p, _c_p]),
@@ -457,6 +465,73 @@ def decode_step_absmax(q, k_cache, v_cache, codes, L: int, k: int, ratio: float,
         _dtype_code(k_cache), B, Hq, Hkv, d, Lmax, L, k, float(ratio), int(bool(shared)),
         _dev(ws, "workspace"), ws.numel(), idx_ptr, _dev(out, "out"), _stream(stream)),
         "adamas_decode_step_absmax")
+    return out
+
+
+# ------------------------------------------------ context-parallel steps
+PART_STRIDE = 132      # floats per exported softmax partial: m, l, 0, 0, acc[128]
+
+
+def cp_hist_shape(B: int, Hq: int, Hkv: int, shared: bool = False):
+    n = int(lib().adamas_cp_hist_elems(B, Hq, Hkv, int(bool(shared))))
+    if n == 0:
+        raise AdamasError(ERR_INVALID_ARG, "adamas_cp_hist_elems")
+    rows = B * (Hkv if shared else Hq)
+    return (B, rows // B, n // rows)
+
+
+def cp_workspace(B: int, Hq: int, Hkv: int, L: int, k: int, shared: bool = False, device="cuda",
+                 stream=None):
+    """A zero-filled workspace for one rank's context-parallel steps (L: its positions)."""
+    n = int(lib().adamas_cp_workspace_bytes(B, Hq, Hkv, HEAD_DIM, L, k, int(bool(shared))))
+    if n == 0:
+        raise AdamasError(ERR_INVALID_ARG, "adamas_cp_workspace_bytes")
+    return init_workspace(torch.empty(n, dtype=torch.uint8, device=device), stream)
+
+
+def cp_histograms(q, codes, L: int, k: int, t: float, ws, shared: bool = False, hist_out=None,
+                  stream=None):
+    """Phase 1 on this rank's slice: cumulative hist [B, rows, bins] int32 (uint32
+    counts of distances <= bin)."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = codes.shape
+    if hist_out is None:
+        hist_out = torch.empty(cp_hist_shape(B, Hq, Hkv, shared), dtype=torch.int32,
+                               device=q.device)
+    _check(lib().adamas_cp_histograms(_dev(q, "q"), _dev(codes, "codes"), _dtype_code(q), B, Hq,
+                                      Hkv, d, Lmax, L, k, float(t), int(bool(shared)),
+                                      _dev(ws, "workspace"), ws.numel(), _dev(hist_out, "hist"),
+                                      _stream(stream)), "adamas_cp_histograms")
+    return hist_out
+
+
+def cp_attend(q, k_cache, v_cache, codes, L: int, L_total: int, pos_offset: int, k: int,
+              t: float, hist_all, rank: int, ws, shared: bool = False, idx_out=None,
+              partial_out=None, stream=None):
+    """Phase 2 on this rank's slice, given every rank's cumulative histograms
+    hist_all [world, B, rows, bins]: partial [B, Hq, 132] float32."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if partial_out is None:
+        partial_out = torch.empty((B, Hq, PART_STRIDE), dtype=torch.float32, device=q.device)
+    idx_ptr = None if idx_out is None else _dev(idx_out, "idx_out")
+    _check(lib().adamas_cp_attend(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                  _dev(codes, "codes"), _dtype_code(k_cache), B, Hq, Hkv, d, Lmax,
+                                  L, L_total, pos_offset, k, float(t), int(bool(shared)),
+                                  _dev(hist_all, "hist_all"), hist_all.shape[0], rank,
+                                  _dev(ws, "workspace"), ws.numel(), idx_ptr,
+                                  _dev(partial_out, "partial"), _stream(stream)),
+           "adamas_cp_attend")
+    return partial_out
+
+
+def cp_combine(partials_all, out=None, stream=None):
+    """partials_all [world, B, Hq, 132] -> out [B, Hq, 128] float32."""
+    world, B, Hq, _ = partials_all.shape
+    if out is None:
+        out = torch.empty((B, Hq, HEAD_DIM), dtype=torch.float32, device=partials_all.device)
+    _check(lib().adamas_cp_combine(_dev(partials_all, "partials"), world, B, Hq, _dev(out, "out"),
+                                   _stream(stream)), "adamas_cp_combine")
     return out
 
 

@@ -485,6 +485,88 @@ adamas_status adamas_select_topk_paged(const uint8_t* qcodes, const uint8_t* cod
 }
 
 
+size_t adamas_cp_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k, int shared) {
+  if (check_decode_sizes(B, Hq, Hkv, d, L, L, k) != ADAMAS_OK || (shared != 0 && shared != 1))
+    return 0;
+  return cp_workspace_bytes(B, Hq, Hkv, L, k, shared != 0);
+}
+
+size_t adamas_cp_hist_elems(int B, int Hq, int Hkv, int shared) {
+  if (B <= 0 || !good_group(Hq, Hkv) || (shared != 0 && shared != 1)) return 0;
+  const int G = Hq / Hkv;
+  return size_t(B) * (shared ? Hkv : Hq) * selection_bins(G, shared != 0);
+}
+
+adamas_status adamas_cp_histograms(const void* q, const uint8_t* codes, adamas_dtype dt, int B,
+                                   int Hq, int Hkv, int d, int64_t Lmax, int64_t L, int k,
+                                   float t, int shared, void* workspace, size_t ws_bytes,
+                                   uint32_t* hist_out, cudaStream_t stream) {
+  if (!q || !codes || !workspace || !hist_out || (shared != 0 && shared != 1))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (!good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(q, 16) || !aligned(codes, 16) || !aligned(workspace, 256) ||
+      !aligned(hist_out, 4))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < cp_workspace_bytes(B, Hq, Hkv, L, k, shared != 0))
+    return ADAMAS_ERR_INVALID_ARG;
+  CpArgs cpa = {};
+  cpa.phase = 1;
+  cpa.L_total = L;
+  cpa.hist_out = hist_out;
+  return from_cuda(launch_decode(q, nullptr, nullptr, nullptr, codes, dt, B, Hq, Hkv,
+                                 contiguous(Lmax), L, k, t, workspace, nullptr, nullptr,
+                                 shared != 0, p, stream, 0.0f, &cpa));
+}
+
+adamas_status adamas_cp_attend(const void* q, const void* k_cache, const void* v_cache,
+                               const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
+                               int d, int64_t Lmax, int64_t L, int64_t L_total,
+                               int64_t pos_offset, int k, float t, int shared,
+                               const uint32_t* hist_all, int world, int rank, void* workspace,
+                               size_t ws_bytes, int32_t* idx_out, float* partial_out,
+                               cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !codes || !hist_all || !workspace || !partial_out ||
+      (shared != 0 && shared != 1) || world < 1 || rank < 0 || rank >= world)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (!good_dtype(dt) || !good_t(t)) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (pos_offset < 0 || L_total < pos_offset + L || L_total > INT32_MAX)
+    return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(codes, 16) ||
+      !aligned(hist_all, 4) || !aligned(partial_out, 16) || !aligned(workspace, 256) ||
+      (idx_out && !aligned(idx_out, 4)))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p))
+    return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < cp_workspace_bytes(B, Hq, Hkv, L, k, shared != 0))
+    return ADAMAS_ERR_INVALID_ARG;
+  CpArgs cpa = {};
+  cpa.phase = 2;
+  cpa.L_total = L_total;
+  cpa.pos_offset = pos_offset;
+  cpa.hist_all = hist_all;
+  cpa.world = world;
+  cpa.rank = rank;
+  cpa.partial_out = partial_out;
+  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
+                                 contiguous(Lmax), L, k, t, workspace, idx_out, nullptr,
+                                 shared != 0, p, stream, 0.0f, &cpa));
+}
+
+adamas_status adamas_cp_combine(const float* partials_all, int world, int B, int Hq, float* out,
+                                cudaStream_t stream) {
+  if (!partials_all || !out || world < 1 || B <= 0 || Hq <= 0) return ADAMAS_ERR_INVALID_ARG;
+  if (!aligned(partials_all, 16) || !aligned(out, 16)) return ADAMAS_ERR_INVALID_ARG;
+  return from_cuda(launch_cp_combine(partials_all, world, int64_t(B) * Hq, out, stream));
+}
+
 adamas_status adamas_select_topk_shared(const uint8_t* qcodes, const uint8_t* codes, int B,
                                         int Hq, int Hkv, int64_t Lmax, int64_t L, int k,
                                         void* workspace, size_t ws_bytes, int32_t* idx_out,

@@ -498,6 +498,7 @@ struct Plan {
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
                                     int page_shift, Plan& p);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k);
+size_t cp_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k, bool shared);
 size_t decode_workspace_error_offset();
 // Where a unit's positions live.  Contiguous caches: unit (b, kv head) owns rows
 // [unit * Lmax, unit * Lmax + L).  Paged caches (block_table != nullptr): position p
@@ -512,11 +513,28 @@ struct CacheLayout {
   int page_shift = 0;
   int64_t num_pages = 0;
 };
+// One rank's part of a context-parallel step: the rank holds positions
+// [pos_offset, pos_offset + L) of a context of L_total positions.
+struct CpArgs {
+  int phase;               // 1: export distance histograms; 2: select + attend + export partials
+  int64_t L_total;
+  int64_t pos_offset;
+  uint32_t* hist_out;      // phase 1: [B][rows][bins] cumulative counts over the slice
+                           //          (rows: Hq, or Hkv for shared selection)
+  const uint32_t* hist_all;  // phase 2: [world][B][rows][bins], every rank's hist_out
+  int world, rank;
+  float* partial_out;      // phase 2: [B][Hq][kPartStride]: m (log2 domain), l, 0, 0, acc[128]
+};
 cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
                           const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
                           int32_t* idx_out, float* out, bool shared, const Plan& p,
-                          cudaStream_t stream, float t_ratio = 0.0f);
+                          cudaStream_t stream, float t_ratio = 0.0f,
+                          const CpArgs* cpa = nullptr);
+// Distance bins of a selection row: 385 per query head, 384 G + 1 for shared selection.
+inline int selection_bins(int G, bool shared) { return shared ? 384 * G + 1 : 3 * kD + 1; }
+cudaError_t launch_cp_combine(const float* partials, int world, int64_t rows, float* out,
+                              cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
                                cudaStream_t stream, const int32_t* ids = nullptr,

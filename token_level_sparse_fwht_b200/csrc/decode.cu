@@ -42,6 +42,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = kThreads;  // keys per bulk copy (16 KiB of codes), one per thread
 constexpr int kMaxStages = 8;    // bulk-copy ring depth (runtime: 1..8, as shared memory allows)
 constexpr int kMaxCluster = 16;  // non-portable cluster size limit
+// kernel flavours: contiguous caches, paged caches, one rank of a context-parallel step
+constexpr int kModeContiguous = 0, kModePaged = 1, kModeCP = 2;
 constexpr int kNCoarse = 30;     // coarse chunks of the D* search (30 x chunk >= bins)
 constexpr int kCoarseRow = 32;   // coarse counts per (CTA, head), padded to 128 B
 constexpr int kRound = kThreads * 32;   // tokens per select round (32 per thread)
@@ -74,6 +76,14 @@ struct DecodeArgs {
   int list_cap;
   int stages;                // bulk-copy ring depth
   int attend;
+  // context-parallel slice (kModeCP): see CpArgs
+  int cp_phase;
+  int64_t L_total, pos_offset;
+  uint32_t* cp_hist_out;
+  uint8_t* cp_scratch;       // per CTA: distances [GS][RS] u16, then cumulative hist [GS][BS]
+  const uint32_t* cp_hist_all;
+  int cp_world, cp_rank;
+  float* cp_partial;
 };
 
 // Selection geometry of one kernel flavour.  Per-head selection (SH = false):
@@ -143,6 +153,12 @@ __host__ __device__ inline SmemLayout layout_of(int R, int list_cap, int CS, int
   return make_layout(G, X::GS, X::BS, X::FW, X::GM, R, list_cap, CS, stages, ptab);
 }
 
+// Bytes a CTA keeps between the two context-parallel phases: its distances and its
+// cumulative histograms (16-byte multiples).
+__host__ __device__ inline size_t cp_scratch_per_cta(int GS, int BS, int R) {
+  return size_t(GS) * dist_stride(R) * 2 + size_t(GS) * BS * 4;
+}
+
 // Page-table entries a CTA stages: the pages its R positions can span.
 __host__ __device__ inline int ptab_entries(int R, int page_shift, bool paged) {
   return paged ? ((R + (1 << page_shift) - 1) >> page_shift) + 1 : 0;
@@ -198,17 +214,19 @@ __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t 
   }
 }
 
-template <int G, bool SH, bool PG, typename T>
+template <int G, bool SH, int MD, typename T>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a) {
   using X = Sel<G, SH>;
   constexpr int GS = X::GS, BS = X::BS, NB = X::NB, CB = X::C, FW = X::FW, GM = X::GM;
+  constexpr bool paged = MD == kModePaged;
+  constexpr bool cp = MD == kModeCP;   // one rank's slice of a context-parallel step
   extern __shared__ __align__(128) uint8_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = a.cluster;
   const int rank = int(cluster.block_rank());
   const int S = a.stages;
   const SmemLayout lo = layout_of<G, SH>(a.keys_per_cta, a.list_cap, CS, S,
-                                         ptab_entries(a.keys_per_cta, a.page_shift, PG));
+                                         ptab_entries(a.keys_per_cta, a.page_shift, MD == kModePaged));
   uint8_t* ring = smem + lo.ring;
   float* part = reinterpret_cast<float*>(smem + lo.ring);           // [CS][G][kPartStride]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
@@ -238,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     }
     L = min(max(Lb, int64_t(0)), a.L);
   }
-  const int keff = int(min(int64_t(a.budget), L));
+  const int keff = int(min(int64_t(a.budget), cp ? a.L_total : L));
   const int R = a.keys_per_cta;
   const int RS = dist_stride(R);
   const int64_t p0 = int64_t(rank) * R;
@@ -251,7 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   // (pool rows number below 2^31: a row is at least 256 bytes); a page id outside
   // [0, num_pages) is an input error: flagged, and page 0 is used instead so that no
   // access leaves the pool.
-  constexpr bool paged = PG;
   const int psh = a.page_shift;
   const int pmask = (1 << psh) - 1;
   const int64_t pfirst = p0 >> psh;
@@ -298,8 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 
   // ---- issue the code copies first: HBM traffic starts before anything else.  The
   // last warp issues them, so the warps that encode the queries are not delayed.
+  // (context-parallel phase 2 reads its distances back from phase 1: no copies)
+  const bool scan_codes = !(cp && a.cp_phase == 2);
   if constexpr (!paged) {
-    if (tid == kThreads - 32) {
+    if (tid == kThreads - 32 && scan_codes) {
       for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
       fence_mbar_init();
       for (int qi = 0; qi < min(nch, S); ++qi) issue_chunk(qi, qi);
@@ -384,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     const uint32_t one = uint32_t(a.keys_per_cta > 0);   // 1, opaque to the compiler
     int slot = 0;
     uint32_t parity = 0;
-    for (int qi = 0; qi < nch; ++qi) {
+    for (int qi = 0; qi < (scan_codes ? nch : 0); ++qi) {
       if constexpr (paged) {
         cp_async_wait_pending(S - 1);   // this thread's copies of chunk qi have landed
         __syncwarp();                   // ... and its warp-mates' (the key it scans)
@@ -462,7 +481,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
     }
   };
-  if constexpr (CB <= 16) {
+  uint8_t* scratch = nullptr;
+  if constexpr (cp) {
+    scratch = a.cp_scratch + size_t(blockIdx.x) * cp_scratch_per_cta(GS, BS, R);
+  }
+  if (cp && a.cp_phase == 2) {
+    // phase 2: this CTA's distances and cumulative histograms, kept by phase 1
+    const uint4* src = reinterpret_cast<const uint4*>(scratch);
+    uint4* dd = reinterpret_cast<uint4*>(dist);
+    const int nd = GS * RS * 2 / 16;
+    for (int i = tid; i < nd; i += kThreads) dd[i] = src[i];
+    uint4* hh = reinterpret_cast<uint4*>(hist);
+    for (int i = tid; i < GS * BS / 4; i += kThreads) hh[i] = src[nd + i];
+    __syncthreads();
+    if (warp < GS) push_coarse(warp, hist[warp * BS + min(CB * lane + CB - 1, NB - 1)]);
+  } else if constexpr (CB <= 16) {
     // 385 bins (per head, or one shared head of G = 1): a warp per selection head,
     // lane l owning bins CB*l .. CB*l + CB-1 in registers
     if (warp < GS) {
@@ -524,6 +557,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 
   cluster.sync();   // cumulative histograms complete; coarse counts delivered
 
+  if constexpr (cp) {
+    if (a.cp_phase == 1) {
+      // context-parallel phase 1: every CTA keeps its distances and cumulative
+      // histograms for phase 2; the unit's cumulative histogram over this rank's
+      // slice (the sum of its CTAs', gathered by rank 0 through distributed shared
+      // memory; the second barrier keeps the peers alive until it has read them)
+      // is exported for the other ranks
+      {
+        uint4* dst = reinterpret_cast<uint4*>(scratch);
+        const uint4* dd = reinterpret_cast<const uint4*>(dist);
+        const int nd = GS * RS * 2 / 16;
+        for (int i = tid; i < nd; i += kThreads) dst[i] = dd[i];
+        const uint4* hh = reinterpret_cast<const uint4*>(hist);
+        for (int i = tid; i < GS * BS / 4; i += kThreads) dst[nd + i] = hh[i];
+      }
+      if (rank == 0) {
+        for (int i = tid; i < GS * NB; i += kThreads) {
+          const int g = i / NB, bin = i % NB;
+          uint32_t c = 0;
+          for (int cc = 0; cc < CS; ++cc) c += cluster.map_shared_rank(hist, cc)[g * BS + bin];
+          a.cp_hist_out[(int64_t(unit) * GS + g) * NB + bin] = c;
+        }
+      }
+      cluster.sync();
+      return;
+    }
+  }
+
   // ---- resolve D*, the count selected in lower-ranked CTAs, and the ties taken.
   // Level 1 (local): the coarse chunk j* where the unit's cumulative count reaches
   // k_eff.  Level 2: each peer's FW-bin window around chunk j* is pulled with
@@ -534,6 +595,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     uint32_t S1 = 0;
     if (lane < kNCoarse) {
       for (int cc = 0; cc < CS; ++cc) S1 += coarse[(cc * GS + g) * kCoarseRow + lane];
+      if constexpr (cp) {   // the other ranks' cumulative counts at the chunk end
+        const int64_t rows = int64_t(a.B) * a.Hkv * GS;
+        const int64_t e = (int64_t(unit) * GS + g) * NB + min(CB * lane + CB - 1, NB - 1);
+#pragma unroll 4
+        for (int w = 0; w < a.cp_world; ++w) {
+          if (w != a.cp_rank) S1 += a.cp_hist_all[int64_t(w) * rows * NB + e];
+        }
+      }
     }
     const uint32_t hit1 = __ballot_sync(0xffffffffu, lane < kNCoarse && S1 >= uint32_t(keff));
     if (lane == 0) jst[g] = __ffs(hit1) - 1;   // exists: chunk 29 ends at the last bin, count L
@@ -569,6 +638,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           const uint32_t x = fine[(cc * GS + g) * FW + off];
           S2 += x;
           if (cc < rank) Sb += x;
+        }
+        if constexpr (cp) {   // other ranks count in the total, lower ranks also come first
+          const int64_t rows = int64_t(a.B) * a.Hkv * GS;
+          const int64_t e = (int64_t(unit) * GS + g) * NB + min(d, NB - 1);
+#pragma unroll 4
+          for (int w = 0; w < a.cp_world; ++w) {
+            if (w == a.cp_rank) continue;
+            const uint32_t x = a.cp_hist_all[int64_t(w) * rows * NB + e];
+            S2 += x;
+            if (w < a.cp_rank) Sb += x;
+          }
         }
       }
       const uint32_t hit2 = __ballot_sync(0xffffffffu, l >= 1 && l < CB + 1 && S2 >= ke);
@@ -701,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           // broken invariant from writing outside the list or the output row
           if (rk < nsel[g] && base[g] + rk < keff) {
             lrow[rk] = static_cast<uint16_t>(r);
-            if (orow) orow[rk] = int32_t(p0 + r);
+            if (orow) orow[rk] = int32_t(a.pos_offset + p0 + r);
           }
           ++rk;
         }
@@ -787,7 +867,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 
   cluster.sync();   // partials are in rank 0; no CTA reads a peer's memory after this
 
-  if (a.attend && rank == 0) {
+  if (cp && a.attend && rank == 0) {
+    // context-parallel phase 2: this rank's partial of every head (log2 domain; a
+    // rank that selected nothing for a head exports m = -inf, l = 0)
+    for (int i = tid; i < G * kD; i += kThreads) {
+      const int gg = i / kD, dim = i % kD;
+      float M = -INFINITY;
+      for (int cc = 0; cc < CS; ++cc) M = fmaxf(M, part[(cc * G + gg) * kPartStride]);
+      float Ls = 0.f, A = 0.f;
+      if (M != -INFINITY) {
+        for (int cc = 0; cc < CS; ++cc) {
+          const float* prow = part + (cc * G + gg) * kPartStride;
+          const float e = exp2f(prow[0] - M);
+          Ls = fmaf(prow[1], e, Ls);
+          A = fmaf(prow[4 + dim], e, A);
+        }
+      }
+      float* pr = a.cp_partial + (int64_t(b) * a.Hq + kvh * G + gg) * kPartStride;
+      if (dim == 0) { pr[0] = M; pr[1] = Ls; pr[2] = 0.f; pr[3] = 0.f; }
+      pr[4 + dim] = A;
+    }
+  } else if (a.attend && rank == 0) {
     for (int i = tid; i < G * kD; i += kThreads) {
       const int gg = i / kD, dim = i % kD;
       float M = -INFINITY;
@@ -816,17 +916,17 @@ static int max_smem_optin(int dev) {
   return v;
 }
 
-template <int G, bool SH, bool PG, typename T>
+template <int G, bool SH, int MD, typename T>
 static cudaError_t prepare_kernel() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     int dev = 0;
     cudaGetDevice(&dev);
-    err = cudaFuncSetAttribute(decode_kernel<G, SH, PG, T>,
+    err = cudaFuncSetAttribute(decode_kernel<G, SH, MD, T>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem_optin(dev));
     if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(decode_kernel<G, SH, PG, T>,
+      err = cudaFuncSetAttribute(decode_kernel<G, SH, MD, T>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   });
   return err;
@@ -834,7 +934,7 @@ static cudaError_t prepare_kernel() {
 
 template <int G, bool SH, typename T>
 static int active_clusters_g(int cs, size_t smem) {
-  if (prepare_kernel<G, SH, false, T>() != cudaSuccess) return 0;
+  if (prepare_kernel<G, SH, kModeContiguous, T>() != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs);
   cfg.blockDim = dim3(kThreads);
@@ -847,7 +947,7 @@ static int active_clusters_g(int cs, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int nclusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, SH, false, T>, &cfg) !=
+  if (cudaOccupancyMaxActiveClusters(&nclusters, decode_kernel<G, SH, kModeContiguous, T>, &cfg) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -944,13 +1044,23 @@ bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bo
                           p);
 }
 
+// Context-parallel workspace: the error word, then every CTA's scratch.
+size_t cp_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k, bool shared) {
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p)) return 0;
+  const int G = Hq / Hkv;
+  const int NB = selection_bins(G, shared);
+  const int BS = (NB + 3) / 4 * 4;
+  return 256 + size_t(p.grid) * cp_scratch_per_cta(shared ? 1 : G, BS, int(p.keys_per_cta));
+}
+
 // The decode workspace only carries the device error word (bounded copy waits).
 size_t decode_workspace_bytes(int, int, int, int64_t, int) { return 256; }
 size_t decode_workspace_error_offset() { return 8; }
 
-template <int G, bool SH, bool PG, typename T>
+template <int G, bool SH, int MD, typename T>
 static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t stream) {
-  const cudaError_t e = prepare_kernel<G, SH, PG, T>();
+  const cudaError_t e = prepare_kernel<G, SH, MD, T>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
@@ -964,32 +1074,32 @@ static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t str
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<G, SH, PG, T>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<G, SH, MD, T>, a);
 }
 
-template <bool SH, bool PG, typename T>
+template <bool SH, int MD, typename T>
 static cudaError_t launch_t(int G, const DecodeArgs& a, const Plan& p, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_g<1, SH, PG, T>(a, p, s);
-    case 2: return launch_g<2, SH, PG, T>(a, p, s);
-    case 4: return launch_g<4, SH, PG, T>(a, p, s);
-    case 8: return launch_g<8, SH, PG, T>(a, p, s);
+    case 1: return launch_g<1, SH, MD, T>(a, p, s);
+    case 2: return launch_g<2, SH, MD, T>(a, p, s);
+    case 4: return launch_g<4, SH, MD, T>(a, p, s);
+    case 8: return launch_g<8, SH, MD, T>(a, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <bool SH, bool PG>
+template <bool SH, int MD>
 static cudaError_t launch_dt(adamas_dtype dt, int G, const DecodeArgs& a, const Plan& p,
                              cudaStream_t s) {
-  if (dt == ADAMAS_F32) return launch_t<SH, PG, float>(G, a, p, s);
-  return launch_t<SH, PG, __nv_bfloat16>(G, a, p, s);
+  if (dt == ADAMAS_F32) return launch_t<SH, MD, float>(G, a, p, s);
+  return launch_t<SH, MD, __nv_bfloat16>(G, a, p, s);
 }
 
 cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, const void* v,
                           const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv,
                           const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
                           int32_t* idx_out, float* out, bool shared, const Plan& p,
-                          cudaStream_t stream, float t_ratio) {
+                          cudaStream_t stream, float t_ratio, const CpArgs* cpa) {
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q; a.qcodes = qcodes; a.k = k; a.v = v; a.codes = codes;
@@ -1010,14 +1120,27 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.keys_per_cta = int(p.keys_per_cta);
   a.list_cap = p.list_cap;
   a.stages = p.stages;
-  a.attend = out != nullptr ? 1 : 0;
-  const bool paged = lay.block_table != nullptr;
+  a.attend = (out != nullptr || (cpa != nullptr && cpa->phase == 2)) ? 1 : 0;
+  a.cp_phase = cpa ? cpa->phase : 0;
+  a.L_total = cpa ? cpa->L_total : L;
+  a.pos_offset = cpa ? cpa->pos_offset : 0;
+  a.cp_hist_out = cpa ? cpa->hist_out : nullptr;
+  a.cp_scratch = cpa ? static_cast<uint8_t*>(ws) + 256 : nullptr;
+  a.cp_hist_all = cpa ? cpa->hist_all : nullptr;
+  a.cp_world = cpa ? cpa->world : 1;
+  a.cp_rank = cpa ? cpa->rank : 0;
+  a.cp_partial = cpa ? cpa->partial_out : nullptr;
+  if (cpa) a.idx_stride = int(std::min<int64_t>(kk, cpa->L_total));
+  const int mode = cpa != nullptr ? kModeCP
+                   : lay.block_table != nullptr ? kModePaged : kModeContiguous;
   if (shared) {
-    return paged ? launch_dt<true, true>(dt, G, a, p, stream)
-                 : launch_dt<true, false>(dt, G, a, p, stream);
+    return mode == kModeCP      ? launch_dt<true, kModeCP>(dt, G, a, p, stream)
+           : mode == kModePaged ? launch_dt<true, kModePaged>(dt, G, a, p, stream)
+                                : launch_dt<true, kModeContiguous>(dt, G, a, p, stream);
   }
-  return paged ? launch_dt<false, true>(dt, G, a, p, stream)
-               : launch_dt<false, false>(dt, G, a, p, stream);
+  return mode == kModeCP      ? launch_dt<false, kModeCP>(dt, G, a, p, stream)
+         : mode == kModePaged ? launch_dt<false, kModePaged>(dt, G, a, p, stream)
+                              : launch_dt<false, kModeContiguous>(dt, G, a, p, stream);
 }
 
 }  // namespace adamas

@@ -28,6 +28,7 @@
 // the CS partials and writes the output.
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include <cooperative_groups.h>
 
@@ -401,9 +402,93 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     }
     const int swz = (tid >> 2) & 1;   // conflict-free 2 x 16 B reads of a 32 B code
     const uint32_t one = uint32_t(a.keys_per_cta > 0);   // 1, opaque to the compiler
+    // the thermometer words of this thread's key in ring slot `sl`
+    const auto load_key = [&](int sl, Therm& kt) {
+      const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t(sl) * kChunk + tid) *
+                                                        kCodeBytes);
+      const uint4 xa = src[swz], xb = src[swz ^ 1];
+      const uint4 x0 = swz ? xb : xa, x1 = swz ? xa : xb;
+      const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      make_therm(wd, kt);
+    };
+    // distances of NK keys (positions r[]; side effects only where valid[]), with the
+    // keys' work in one block so that their dependency chains interleave (the pair
+    // loop below; the one-chunk loop keeps its own branch-guarded body)
+    const auto score_keys = [&](auto nk_tag, const Therm* kt, const int* r, const bool* valid) {
+      constexpr int NK = decltype(nk_tag)::value;
+      uint32_t dsum[NK];
+#pragma unroll
+      for (int u = 0; u < NK; ++u) dsum[u] = 0;   // shared selection: sum over the heads
+#pragma unroll
+      for (int g0 = 0; g0 < G; g0 += GR) {
+        if constexpr (G > 4) {
+#pragma unroll
+          for (int g = 0; g < GR; ++g) {
+            const uint4* s = reinterpret_cast<const uint4*>(qth + (g0 + g) * 12);
+            const uint4 p0v = s[0], p1v = s[1], p2v = s[2];
+            qreg[g].a[0] = p0v.x; qreg[g].a[1] = p0v.y; qreg[g].a[2] = p0v.z; qreg[g].a[3] = p0v.w;
+            qreg[g].a[4] = p1v.x; qreg[g].a[5] = p1v.y; qreg[g].a[6] = p1v.z; qreg[g].a[7] = p1v.w;
+            qreg[g].b[0] = p2v.x; qreg[g].b[1] = p2v.y; qreg[g].b[2] = p2v.z; qreg[g].b[3] = p2v.w;
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < GR; ++g) {
+#pragma unroll
+          for (int u = 0; u < NK; ++u) {
+            const uint32_t dd = therm_dist_csa(kt[u], qreg[g], one);
+            if constexpr (SH) {
+              dsum[u] += dd;
+            } else if (valid[u]) {
+              dist[size_t(g0 + g) * RS + r[u]] = static_cast<uint16_t>(dd);
+              atomicAdd(&hist[(g0 + g) * BS + dd], 1u);
+            }
+          }
+        }
+      }
+      if constexpr (SH) {
+#pragma unroll
+        for (int u = 0; u < NK; ++u) {
+          if (valid[u]) {
+            dist[r[u]] = static_cast<uint16_t>(dsum[u]);
+            atomicAdd(&hist[dsum[u]], 1u);
+          }
+        }
+      }
+    };
+    using Two = std::integral_constant<int, 2>;
     int slot = 0;
     uint32_t parity = 0;
-    for (int qi = 0; qi < (scan_codes ? nch : 0); ++qi) {
+    int qi = 0;
+    if constexpr (!paged && G <= 2) {
+      // one or two heads per key leave each key's chain short and latency-bound: two
+      // chunks per iteration while the ring holds at least four, their keys scored
+      // together (the next copies are issued once both are consumed).  With four or
+      // more heads the heads already interleave and the popcount pipe is the limit.
+      if (S >= 4) {
+        for (; qi + 1 < (scan_codes ? nch : 0); qi += 2) {
+          int slot2 = slot + 1;
+          uint32_t par2 = parity;
+          if (slot2 == S) { slot2 = 0; par2 ^= 1u; }
+          mbar_wait_bounded(&mbar[slot], parity, a.err);
+          mbar_wait_bounded(&mbar[slot2], par2, a.err);
+          Therm kt[2];
+          load_key(slot, kt[0]);
+          load_key(slot2, kt[1]);
+          const int r[2] = {qi * kChunk + tid, (qi + 1) * kChunk + tid};
+          const bool valid[2] = {r[0] < n, r[1] < n};
+          score_keys(Two{}, kt, r, valid);
+          if (nch > S) __syncthreads();
+          if (tid == kThreads - 32) {
+            if (qi + S < nch) issue_chunk(qi + S, slot);
+            if (qi + 1 + S < nch) issue_chunk(qi + 1 + S, slot2);
+          }
+          slot = slot2 + 1;
+          parity = par2;
+          if (slot == S) { slot = 0; parity ^= 1u; }
+        }
+      }
+    }
+    for (; qi < (scan_codes ? nch : 0); ++qi) {
       if constexpr (paged) {
         cp_async_wait_pending(S - 1);   // this thread's copies of chunk qi have landed
         __syncwarp();                   // ... and its warp-mates' (the key it scans)
@@ -412,13 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
       const int r = qi * kChunk + tid;
       if (r < n) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            ring + (size_t(slot) * kChunk + tid) * kCodeBytes);
-        const uint4 xa = src[swz], xb = src[swz ^ 1];
-        const uint4 x0 = swz ? xb : xa, x1 = swz ? xa : xb;
-        const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         Therm kt;
-        make_therm(wd, kt);
+        load_key(slot, kt);
         uint32_t dsum = 0;   // shared selection: sum of the G heads' distances
 #pragma unroll
         for (int g0 = 0; g0 < G; g0 += GR) {

@@ -27,7 +27,9 @@
 // shared memory of cluster rank 0; after a second cluster barrier rank 0 merges
 // the CS partials and writes the output.
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include <cooperative_groups.h>
@@ -358,7 +360,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       qc[g * kCodeBytes + lane] = a.qcodes[(int64_t(b) * a.Hq + h) * kCodeBytes + lane];
     } else {
       float v[4];
-      load4(static_cast<const T*>(a.q) + (int64_t(b) * a.Hq + h) * kD, lane, v);
+      const T* qsrc = static_cast<const T*>(a.q) + (int64_t(b) * a.Hq + h) * kD;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // 16-byte loads by lanes 0-15 (q may live in mapped host memory, where
+        // fewer, wider requests matter), redistributed to 4 elements per lane
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (lane < 16) x = __ldg(reinterpret_cast<const uint4*>(qsrc) + lane);
+        const int from = lane >> 1;
+        const uint32_t w0 = __shfl_sync(0xffffffffu, x.x, from);
+        const uint32_t w1 = __shfl_sync(0xffffffffu, x.y, from);
+        const uint32_t w2 = __shfl_sync(0xffffffffu, x.z, from);
+        const uint32_t w3 = __shfl_sync(0xffffffffu, x.w, from);
+        bf16x2_to_f32((lane & 1) ? w2 : w0, v[0], v[1]);
+        bf16x2_to_f32((lane & 1) ? w3 : w1, v[2], v[3]);
+      } else {
+        load4(qsrc, lane, v);
+      }
       float* qrow = qf + g * kD + 4 * lane;
       qrow[0] = v[0]; qrow[1] = v[1]; qrow[2] = v[2]; qrow[3] = v[3];
       qc[g * kCodeBytes + lane] =
@@ -968,20 +985,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       pr[4 + dim] = A;
     }
   } else if (a.attend && rank == 0) {
-    for (int i = tid; i < G * kD; i += kThreads) {
-      const int gg = i / kD, dim = i % kD;
+    // four coordinates per thread: 16-byte partial reads and one 16-byte output store
+    // (out may live in mapped host memory, where fewer, wider requests matter)
+    for (int i = tid; i < G * (kD / 4); i += kThreads) {
+      const int gg = i / (kD / 4), d4 = 4 * (i % (kD / 4));
       float M = -INFINITY;
       for (int cc = 0; cc < CS; ++cc) M = fmaxf(M, part[(cc * G + gg) * kPartStride]);
       if (M == -INFINITY) M = 0.f;   // every split empty (length 0): all terms below are 0
-      float Ls = 0.f, A = 0.f;
+      float Ls = 0.f;
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int cc = 0; cc < CS; ++cc) {
         const float* prow = part + (cc * G + gg) * kPartStride;
         const float e = exp2f(prow[0] - M);     // empty split: m = -inf -> 0
+        const float4 x = *reinterpret_cast<const float4*>(prow + 4 + d4);
         Ls = fmaf(prow[1], e, Ls);
-        A = fmaf(prow[4 + dim], e, A);
+        A.x = fmaf(x.x, e, A.x);
+        A.y = fmaf(x.y, e, A.y);
+        A.z = fmaf(x.z, e, A.z);
+        A.w = fmaf(x.w, e, A.w);
       }
       // an empty sequence (length 0) selects nothing: its output is zero
-      a.out[(int64_t(b) * a.Hq + kvh * G + gg) * kD + dim] = Ls > 0.f ? A / Ls : 0.f;
+      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+      *reinterpret_cast<float4*>(a.out + (int64_t(b) * a.Hq + kvh * G + gg) * kD + d4) =
+          make_float4(A.x * inv, A.y * inv, A.z * inv, A.w * inv);
     }
   }
 }
@@ -1112,6 +1138,23 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
   return found && p.grid > 0 && int64_t(p.grid) == U * p.cluster && U * p.cluster < (1ll << 31);
 }
 
+namespace {
+// Plans are memoised per device and problem: making one queries the cluster
+// occupancy of every candidate cluster size, far more host time than a launch.
+struct PlanKey {
+  int dev, B, Hq, Hkv, k, page_shift;
+  int64_t L;
+  bool shared;
+  bool operator<(const PlanKey& o) const {
+    return std::tie(dev, B, Hq, Hkv, k, page_shift, L, shared) <
+           std::tie(o.dev, o.B, o.Hq, o.Hkv, o.k, o.page_shift, o.L, o.shared);
+  }
+};
+std::mutex g_plan_mutex;
+std::map<PlanKey, std::pair<bool, Plan>> g_plans;
+constexpr size_t kMaxPlans = 4096;
+}  // namespace
+
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
                                     int page_shift, Plan& p) {
   int dev = 0;
@@ -1120,8 +1163,18 @@ bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bo
     // no device visible: plan for a 148-SM part with the sm_100 shared-memory cap
     return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, 148, 232448, false, p);
   }
-  return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, sms, max_smem_optin(dev), true,
-                          p);
+  const PlanKey key{dev, B, Hq, Hkv, k, page_shift, L, shared};
+  std::lock_guard<std::mutex> lock(g_plan_mutex);
+  const auto it = g_plans.find(key);
+  if (it != g_plans.end()) {
+    p = it->second.second;
+    return it->second.first;
+  }
+  const bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, sms,
+                                   max_smem_optin(dev), true, p);
+  if (g_plans.size() >= kMaxPlans) g_plans.clear();
+  g_plans.emplace(key, std::make_pair(ok, p));
+  return ok;
 }
 
 // Context-parallel workspace: the error word, then every CTA's scratch.

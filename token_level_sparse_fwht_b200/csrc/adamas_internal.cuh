@@ -493,6 +493,7 @@ struct Plan {
   int list_cap;          // selected-position slots per head per CTA
   int stages;            // bulk-copy ring depth
   size_t smem;           // dynamic shared memory bytes
+  int64_t l2_bytes;      // device L2 capacity (0: unknown)
 };
 // page_shift: log2(page size) for paged caches, -1 for contiguous caches.
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,

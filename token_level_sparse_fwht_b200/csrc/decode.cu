@@ -79,6 +79,7 @@ struct DecodeArgs {
   int list_cap;
   int stages;                // bulk-copy ring depth
   int attend;
+  int prefetch;              // pull rows below D* into L2 during the select
   // context-parallel slice (kModeCP): see CpArgs
   int cp_phase;
   int64_t L_total, pos_offset;
@@ -838,8 +839,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         eqm[g] &= valid;
         cnt[g] = (uint32_t(__popc(ltm[g])) << 16) | uint32_t(__popc(eqm[g]));
         // tokens below D* are selected whatever the tie rule decides: start pulling
-        // their K/V rows into L2 now, so the gather finds them there
-        if (a.attend) {
+        // their K/V rows into L2 now, so the gather finds them there (when the step's
+        // selected rows fit in 3/4 of the L2; beyond that the prefetches evict each
+        // other and only add work)
+        if (a.attend && a.prefetch) {
           uint32_t m = ltm[g];
           while (m) {
             const int i = __ffs(m) - 1;
@@ -1133,6 +1136,7 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
       p.stages = stages;
       p.smem = smem;
       p.waves = int(waves);
+      p.l2_bytes = 0;
     }
   }
   return found && p.grid > 0 && int64_t(p.grid) == U * p.cluster && U * p.cluster < (1ll << 31);
@@ -1172,6 +1176,12 @@ bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bo
   }
   const bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, sms,
                                    max_smem_optin(dev), true, p);
+  int l2 = 0;
+  if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
+    cudaGetLastError();
+    l2 = 0;
+  }
+  p.l2_bytes = l2;
   if (g_plans.size() >= kMaxPlans) g_plans.clear();
   g_plans.emplace(key, std::make_pair(ok, p));
   return ok;
@@ -1254,6 +1264,12 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.list_cap = p.list_cap;
   a.stages = p.stages;
   a.attend = (out != nullptr || (cpa != nullptr && cpa->phase == 2)) ? 1 : 0;
+  {
+    // selected K and V bytes of the whole step (rows gathered once per selection row)
+    const int64_t rows = int64_t(B) * (shared ? Hkv : Hq) * a.idx_stride;
+    const int64_t sel_bytes = rows * 2 * kD * (dt == ADAMAS_F32 ? 4 : 2);
+    a.prefetch = (p.l2_bytes <= 0 || 4 * sel_bytes <= 3 * p.l2_bytes) ? 1 : 0;
+  }
   a.cp_phase = cpa ? cpa->phase : 0;
   a.L_total = cpa ? cpa->L_total : L;
   a.pos_offset = cpa ? cpa->pos_offset : 0;

@@ -246,10 +246,15 @@ __device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane
 
 // --------------------------------------------------------- code arithmetic
 // Thermometer form of a word of 16 packed codes: for code c = 2h + l the field
-// becomes (odd, even) = ([c >= 3], [c >= 1]).
-__device__ __forceinline__ uint32_t therm13(uint32_t w) {
+// becomes (odd, even) = ([c >= 3], [c >= 1]).  Only c = 2 (binary 10) changes, to
+// 01: subtracting d = h & ~l at the even bit does it without borrows, as one
+// integer multiply-add w + d * neg1 (neg1 = 0xffffffff, held in a register the
+// compiler cannot fold) on the FMA pipe, leaving the logic pipe one op lighter.
+__device__ __forceinline__ uint32_t therm13(uint32_t w, uint32_t neg1) {
   const uint32_t d = (w >> 1) & ~w & 0x55555555u;      // h & ~l, at the even bit
-  return w ^ (d * 3u);   // d has even bits only: d * 3 = d | d << 1 (on the FMA pipe)
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(d), "r"(neg1), "r"(w));
+  return r;
 }
 // [c >= 2] of two words, the first at even bits, the second at odd bits.
 __device__ __forceinline__ uint32_t therm2(uint32_t w0, uint32_t w1) {
@@ -262,9 +267,11 @@ struct Therm {
   uint32_t b[4];
 };
 
-__device__ __forceinline__ void make_therm(const uint32_t w[8], Therm& t) {
+// `one` is 1 at run time, opaque to the compiler (see therm_dist_csa).
+__device__ __forceinline__ void make_therm(const uint32_t w[8], Therm& t, uint32_t one) {
+  const uint32_t neg1 = 0u - one;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) t.a[i] = therm13(w[i]);
+  for (int i = 0; i < 8; ++i) t.a[i] = therm13(w[i], neg1);
 #pragma unroll
   for (int i = 0; i < 4; ++i) t.b[i] = therm2(w[2 * i], w[2 * i + 1]);
 }
@@ -282,10 +289,13 @@ __device__ __forceinline__ uint32_t therm_dist(const Therm& k, const Therm& q) {
   return s0 + s1 + s2;
 }
 
-// Same distance with one carry-save level: the 12 XOR words are added bitwise three
-// at a time (sum word = a^b^c, carry word = majority(a,b,c), both single LOP3s),
-// so 8 popcounts replace 12.  POPC issues at a quarter of the integer-logic rate on
-// sm_100, so this moves work from the saturated popcount pipe to the logic pipe.
+// Same distance with two carry-save levels.  The 12 XOR words are added bitwise three
+// at a time (sum word = a^b^c, carry word = majority(a,b,c), both single LOP3s) into
+// four weight-1 and four weight-2 words; three of each are added again, leaving
+// weight-1 words O and o3, weight-2 words T1, T2 and t3, and one weight-4 word F:
+// 6 popcounts replace 12.  POPC issues at a quarter of the integer-logic rate on
+// sm_100, so this moves work from the popcount pipe to the logic pipe, where the
+// thermometer words' multiply-adds (therm13) made room.
 __device__ __forceinline__ uint32_t therm_dist_csa(const Therm& k, const Therm& q,
                                                    uint32_t one) {
   uint32_t x[12];
@@ -296,17 +306,25 @@ __device__ __forceinline__ uint32_t therm_dist_csa(const Therm& k, const Therm& 
   // The sums run as integer multiply-adds with a multiplier the compiler cannot
   // fold (one == 1 at run time), which keeps them on the FMA pipe and leaves the
   // integer-logic pipe, the scan's bottleneck, to the XOR / carry-save work.
-  uint32_t ones = 0, twos = 0;
+  uint32_t o[4], tw[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t a = x[3 * j], b = x[3 * j + 1], c = x[3 * j + 2];
-    asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(ones) : "r"(uint32_t(__popc(a ^ b ^ c))), "r"(one));
-    asm("mad.lo.u32 %0, %1, %2, %0;"
-        : "+r"(twos)
-        : "r"(uint32_t(__popc((a & b) | (c & (a | b))))), "r"(one));
+    o[j] = a ^ b ^ c;
+    tw[j] = (a & b) | (c & (a | b));
   }
+  const uint32_t O = o[0] ^ o[1] ^ o[2];
+  const uint32_t T1 = (o[0] & o[1]) | (o[2] & (o[0] | o[1]));
+  const uint32_t T2 = tw[0] ^ tw[1] ^ tw[2];
+  const uint32_t F = (tw[0] & tw[1]) | (tw[2] & (tw[0] | tw[1]));
+  // sum = popc(O) + popc(o3) + 2 (popc(T1) + popc(T2) + popc(t3)) + 4 popc(F)
+  uint32_t s1 = uint32_t(__popc(O)), s2 = uint32_t(__popc(T1));
+  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s1) : "r"(uint32_t(__popc(o[3]))), "r"(one));
+  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s2) : "r"(uint32_t(__popc(T2))), "r"(one));
+  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s2) : "r"(uint32_t(__popc(tw[3]))), "r"(one));
   uint32_t r;
-  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(twos), "r"(one + one), "r"(ones));
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(s2), "r"(one + one), "r"(s1));
+  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(r) : "r"(uint32_t(__popc(F))), "r"(4u * one));
   return r;
 }
 

@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
 #pragma unroll
     for (int i = 0; i < 8; ++i) wd[i] = wq[i];
     Therm th;
-    make_therm(wd, th);
+    make_therm(wd, th, uint32_t(a.keys_per_cta > 0));
     uint32_t* dst = qth + tid * 12;
 #pragma unroll
     for (int i = 0; i < 8; ++i) dst[i] = th.a[i];
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       const uint4 xa = src[swz], xb = src[swz ^ 1];
       const uint4 x0 = swz ? xb : xa, x1 = swz ? xa : xb;
       const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      make_therm(wd, kt);
+      make_therm(wd, kt, one);
     };
     // distances of NK keys (positions r[]; side effects only where valid[]), with the
     // keys' work in one block so that their dependency chains interleave (the pair

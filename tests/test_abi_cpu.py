@@ -247,3 +247,15 @@ def test_context_parallel_workspace_size():
     assert n == 256 + p["ctas"] * per_cta
     assert ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 128, 16384, 128, 2) == 0
     assert ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 64, 16384, 128, 0) == 0
+
+
+def test_scratch_distance_plan_workspace():
+    # many units over a long context: the plan keeps each CTA's distances (u16 per key
+    # and head) in the workspace, so fewer, longer CTAs run in one wave
+    B, Hq, Hkv, L, k = 4, 32, 8, 131072, 1024
+    p = ad.decode_plan(B, Hq, Hkv, L, k)
+    n = ad.decode_workspace_bytes(B, Hq, Hkv, L, k)
+    stride = (p["tokens_per_cta"] + 7) // 8 * 8
+    assert n == 256 + p["ctas"] * (Hq // Hkv) * stride * 2
+    assert p["ctas"] <= 148                                      # one wave
+    assert ad.decode_workspace_bytes(1, 32, 8, 32768, 128) == 256   # fits on chip

@@ -199,3 +199,49 @@ def test_prepared_decode_host_call():
         call()
         torch.cuda.synchronize()
         assert torch.equal(out_host, want)
+
+
+def test_long_context_plan_with_scratch_distances_select_exact():
+    """Batch 4 x 8 kv heads at 128K: the plan keeps each CTA's distances in workspace
+    scratch (fewer, longer CTAs in one wave).  Random codes: sampled rows bit-exact."""
+    B, Hq, Hkv, L, k = 4, 32, 8, 131072, 1024
+    assert ad.decode_workspace_bytes(B, Hq, Hkv, L, k) > 256      # the scratch plan
+    rng = np.random.default_rng(77)
+    qc = rng.integers(0, 256, size=(B, Hq, 32), dtype=np.uint8)
+    kc = rng.integers(0, 256, size=(B, Hkv, L, 32), dtype=np.uint8)
+    ws = ad.decode_workspace(B, Hq, Hkv, L, k)
+    idx = ad.select_topk(upload(qc), upload(kc), L, k, ws)
+    torch.cuda.synchronize()
+    ad.check_workspace(ws)
+    idx = idx.cpu().numpy()
+    uq, G = oracle.unpack_codes(qc), Hq // Hkv
+    for b, h in [(0, 0), (1, 13), (2, 22), (3, 31)]:
+        d = oracle.manhattan(uq[b, h], oracle.unpack_codes(kc[b, h // G]))
+        assert np.array_equal(idx[b, h], oracle.select_topk(d, k)), (b, h)
+
+
+def test_long_context_plan_with_scratch_distances_decode():
+    """The same plan through the fused step: the oracle's key codes for two sampled kv
+    heads (the GPU encoder's elsewhere), their query heads checked against the oracle."""
+    w = WORKLOADS[5].scaled(layers=1)
+    inp = generate(w, "cuda")
+    assert ad.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.L, 1024) > 256
+    codes = torch.empty(inp.k_cache.shape[:-1] + (32,), dtype=torch.uint8, device="cuda")
+    ad.encode_keys(inp.k_cache, codes, 0, w.L, inp.t)
+    sampled = [(0, 1), (3, 6)]
+    kcs = {}
+    for b, kvh in sampled:
+        kcs[(b, kvh)] = oracle_codes(inp.k_cache[b, kvh].cpu(), inp.t)
+        codes[b, kvh] = upload(kcs[(b, kvh)])
+    ws = ad.decode_workspace(w.B, w.Hq, w.Hkv, w.L, 1024)
+    idx = torch.empty((w.B, w.Hq, 1024), dtype=torch.int32, device="cuda")
+    out = ad.decode_step(inp.q, inp.k_cache, inp.v_cache, codes, w.L, 1024, inp.t, ws,
+                         idx_out=idx)
+    torch.cuda.synchronize()
+    ad.check_workspace(ws)
+    idx, out, q = idx.cpu().numpy(), out.cpu().numpy(), f64(inp.q)
+    G = w.G
+    for b, kvh in sampled:
+        K, V = f64(inp.k_cache[b, kvh]), f64(inp.v_cache[b, kvh])
+        for h in range(kvh * G, (kvh + 1) * G):
+            check_decode_head(idx[b, h], out[b, h], q[b, h], K, V, kcs[(b, kvh)], 1024, inp.t)

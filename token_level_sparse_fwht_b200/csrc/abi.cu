@@ -196,7 +196,7 @@ adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, cons
       !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p))
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p, shared == 0))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
@@ -237,7 +237,7 @@ adamas_status plan_common(bool shared, int B, int Hq, int Hkv, int d, int64_t L,
   const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, L, L, k);
   if (s != ADAMAS_OK) return s;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p, !shared))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ctas) *ctas = p.grid;
   if (cluster) *cluster = p.cluster;
@@ -259,7 +259,7 @@ adamas_status decode_common(bool shared, const void* q, const void* k_cache,
       !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p, !shared))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
@@ -285,7 +285,7 @@ adamas_status decode_host_common(bool shared, const void* q_host, void* q_dev,
       (idx_out && !aligned(idx_out, 4)))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p, !shared))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   // Page-locked host buffers are mapped into the device's address space: then the
@@ -320,7 +320,7 @@ adamas_status select_common(bool shared, const uint8_t* qcodes, const uint8_t* c
       !aligned(idx_out, 4))
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p))
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, -1, p, !shared))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(nullptr, qcodes, nullptr, nullptr, codes, ADAMAS_BF16, B, Hq,
@@ -368,7 +368,8 @@ adamas_status layout_common(bool shared, const void* q, const uint8_t* qcodes, c
     return ADAMAS_ERR_INVALID_ARG;
   Plan p;
   const int page_shift = lay.block_table != nullptr ? lay.page_shift : -1;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, page_shift, p))
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared, page_shift, p,
+                                      !shared && page_shift < 0))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
   return from_cuda(launch_decode(q, qcodes, kc, vc, codes, select_only ? ADAMAS_BF16 : dt, B, Hq,

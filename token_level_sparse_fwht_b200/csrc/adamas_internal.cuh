@@ -512,10 +512,12 @@ struct Plan {
   int stages;            // bulk-copy ring depth
   size_t smem;           // dynamic shared memory bytes
   int64_t l2_bytes;      // device L2 capacity (0: unknown)
+  bool dist_global;      // distances in workspace scratch, not shared memory
 };
-// page_shift: log2(page size) for paged caches, -1 for contiguous caches.
+// page_shift: log2(page size) for paged caches, -1 for contiguous caches.  allow_gd:
+// the plan may keep distances in workspace scratch (contiguous per-head kernels).
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
-                                    int page_shift, Plan& p);
+                                    int page_shift, Plan& p, bool allow_gd = false);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k);
 size_t cp_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k, bool shared);
 size_t decode_workspace_error_offset();

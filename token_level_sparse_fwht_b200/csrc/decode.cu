@@ -45,8 +45,10 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = kThreads;  // keys per bulk copy (16 KiB of codes), one per thread
 constexpr int kMaxStages = 8;    // bulk-copy ring depth (runtime: 1..8, as shared memory allows)
 constexpr int kMaxCluster = 16;  // non-portable cluster size limit
-// kernel flavours: contiguous caches, paged caches, one rank of a context-parallel step
-constexpr int kModeContiguous = 0, kModePaged = 1, kModeCP = 2;
+// kernel flavours: contiguous caches, paged caches, one rank of a context-parallel step,
+// contiguous caches with each CTA's distances in workspace scratch instead of shared
+// memory (per-head selection over long CTA ranges: fewer, longer CTAs in one wave)
+constexpr int kModeContiguous = 0, kModePaged = 1, kModeCP = 2, kModeContigGD = 3;
 constexpr int kNCoarse = 30;     // coarse chunks of the D* search (30 x chunk >= bins)
 constexpr int kCoarseRow = 32;   // coarse counts per (CTA, head), padded to 128 B
 constexpr int kRound = kThreads * 32;   // tokens per select round (32 per thread)
@@ -80,6 +82,7 @@ struct DecodeArgs {
   int stages;                // bulk-copy ring depth
   int attend;
   int prefetch;              // pull rows below D* into L2 during the select
+  uint16_t* dist_scratch;    // kModeContigGD: per CTA [GS][RS] distances (workspace)
   // context-parallel slice (kModeCP): see CpArgs
   int cp_phase;
   int64_t L_total, pos_offset;
@@ -121,7 +124,8 @@ __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / 
 // after the partials: the ring is idle once the scan is over, and rank 0 receives
 // the peers' partials only after the first cluster barrier.
 __host__ __device__ inline SmemLayout make_layout(int G, int GS, int BS, int FW, int GM, int R,
-                                                 int list_cap, int CS, int stages, int ptab) {
+                                                 int list_cap, int CS, int stages, int ptab,
+                                                 bool dist_smem) {
   SmemLayout s;
   size_t o = 0;
   const size_t ring = size_t(stages) * kChunk * kCodeBytes;
@@ -132,7 +136,7 @@ __host__ __device__ inline SmemLayout make_layout(int G, int GS, int BS, int FW,
   s.hist = o;  o = al(o + size_t(GS) * BS * 4, 128);
   s.coarse = o; o = al(o + size_t(CS) * GS * kCoarseRow * 4, 128);   // pushed by the peers
   s.fine = o;  o = al(o + size_t(CS) * GS * FW * 4, 128);            // pulled from the peers
-  s.dist = o;  o = al(o + size_t(GS) * dist_stride(R) * 2, 128);
+  s.dist = o;  o = al(o + (dist_smem ? size_t(GS) * dist_stride(R) * 2 : 0), 128);
   s.list = o;  o = al(o + size_t(GS) * list_cap * 2, 128);
   s.qf = o;    o = al(o + size_t(G) * kD * 4, 128);
   s.qc = o;    o = al(o + size_t(G) * kCodeBytes, 128);
@@ -152,9 +156,9 @@ __host__ __device__ inline SmemLayout make_layout(int G, int GS, int BS, int FW,
 
 template <int G, bool SH>
 __host__ __device__ inline SmemLayout layout_of(int R, int list_cap, int CS, int stages,
-                                                int ptab) {
+                                                int ptab, bool dist_smem = true) {
   using X = Sel<G, SH>;
-  return make_layout(G, X::GS, X::BS, X::FW, X::GM, R, list_cap, CS, stages, ptab);
+  return make_layout(G, X::GS, X::BS, X::FW, X::GM, R, list_cap, CS, stages, ptab, dist_smem);
 }
 
 // Bytes a CTA keeps between the two context-parallel phases: its distances and its
@@ -230,14 +234,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   const int rank = int(cluster.block_rank());
   const int S = a.stages;
   const SmemLayout lo = layout_of<G, SH>(a.keys_per_cta, a.list_cap, CS, S,
-                                         ptab_entries(a.keys_per_cta, a.page_shift, MD == kModePaged));
+                                         ptab_entries(a.keys_per_cta, a.page_shift, MD == kModePaged),
+                                         MD != kModeContigGD);
   uint8_t* ring = smem + lo.ring;
   float* part = reinterpret_cast<float*>(smem + lo.ring);           // [CS][G][kPartStride]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + lo.hist);    // [GS][BS]
   uint32_t* coarse = reinterpret_cast<uint32_t*>(smem + lo.coarse);  // [CS][GS][kCoarseRow]
   uint32_t* fine = reinterpret_cast<uint32_t*>(smem + lo.fine);      // [CS][GS][FW]
-  uint16_t* dist = reinterpret_cast<uint16_t*>(smem + lo.dist);    // [GS][RS]
+  uint16_t* dist;                                                   // [GS][RS]
+  if constexpr (MD == kModeContigGD) {
+    dist = a.dist_scratch + size_t(blockIdx.x) * X::GS * dist_stride(a.keys_per_cta);
+  } else {
+    dist = reinterpret_cast<uint16_t*>(smem + lo.dist);
+  }
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + lo.list);    // [GS][list_cap]
   float* qf = reinterpret_cast<float*>(smem + lo.qf);              // [G][128]
   uint8_t* qc = smem + lo.qc;                                       // [G][32]
@@ -1080,11 +1090,11 @@ static int active_clusters(int G, bool shared, int cs, size_t smem) {
 }
 
 static size_t layout_total(int G, bool shared, int R, int list_cap, int cs, int stages,
-                           int ptab) {
+                           int ptab, bool dist_smem = true) {
 #define ADAMAS_LAYOUT_CASE(GG)                                                        \
   case GG:                                                                            \
-    return shared ? layout_of<GG, true>(R, list_cap, cs, stages, ptab).total          \
-                  : layout_of<GG, false>(R, list_cap, cs, stages, ptab).total;
+    return shared ? layout_of<GG, true>(R, list_cap, cs, stages, ptab, dist_smem).total \
+                  : layout_of<GG, false>(R, list_cap, cs, stages, ptab, dist_smem).total;
   switch (G) {
     ADAMAS_LAYOUT_CASE(1)
     ADAMAS_LAYOUT_CASE(2)
@@ -1099,7 +1109,7 @@ static size_t layout_total(int G, bool shared, int R, int list_cap, int cs, int 
 // whose clusters can be scheduled), the one with the least modelled time
 // waves x (per-key scan cost x keys per CTA + fixed per-wave latency).
 bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int page_shift,
-                      int sms, int smem_cap, bool query_device, Plan& p) {
+                      bool allow_gd, int sms, int smem_cap, bool query_device, Plan& p) {
   const int G = Hq / Hkv;
   const int64_t U = int64_t(B) * Hkv;
   const int64_t k_eff = std::min<int64_t>(k, L);
@@ -1111,32 +1121,37 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
     if (cs > 1 && (L + R - 1) / R < cs) continue;  // an all-empty tail CTA: use fewer
     const int list_cap = int(std::max<int64_t>(1, std::min<int64_t>(R, k_eff)));
     const int64_t nchunks = (R + kChunk - 1) / kChunk;
-    int stages = int(std::min<int64_t>(kMaxStages, std::max<int64_t>(1, nchunks)));
     const int ptab = ptab_entries(int(R), page_shift, page_shift >= 0);
-    while (stages > 1 &&
-           layout_total(G, shared, int(R), list_cap, cs, stages, ptab) > size_t(smem_cap))
-      --stages;
-    const size_t smem = layout_total(G, shared, int(R), list_cap, cs, stages, ptab);
-    if (smem > size_t(smem_cap)) continue;
-    int conc_clusters = sms / cs;
-    if (query_device) conc_clusters = active_clusters(G, shared, cs, smem);
-    if (conc_clusters < 1) continue;
-    const int64_t total = U * cs;
-    const int64_t conc = int64_t(conc_clusters) * cs;
-    const int64_t waves = (total + conc - 1) / conc;
-    const double per_key_ns = 0.45 * G + 0.35;
-    const double cost = double(waves) * (per_key_ns * double(R) + 6000.0);
-    if (!found || cost < best) {
-      best = cost;
-      found = true;
-      p.grid = int(total);
-      p.cluster = cs;
-      p.keys_per_cta = R;
-      p.list_cap = list_cap;
-      p.stages = stages;
-      p.smem = smem;
-      p.waves = int(waves);
-      p.l2_bytes = 0;
+    // distances in shared memory; or, where allowed, in workspace scratch (their global
+    // stores and reloads cost about 15 % of the scan, modelled below)
+    for (int gd = 0; gd <= (allow_gd ? 1 : 0); ++gd) {
+      int stages = int(std::min<int64_t>(kMaxStages, std::max<int64_t>(1, nchunks)));
+      while (stages > 1 && layout_total(G, shared, int(R), list_cap, cs, stages, ptab, !gd) >
+                               size_t(smem_cap))
+        --stages;
+      const size_t smem = layout_total(G, shared, int(R), list_cap, cs, stages, ptab, !gd);
+      if (smem > size_t(smem_cap)) continue;
+      int conc_clusters = sms / cs;
+      if (query_device) conc_clusters = active_clusters(G, shared, cs, smem);
+      if (conc_clusters < 1) continue;
+      const int64_t total = U * cs;
+      const int64_t conc = int64_t(conc_clusters) * cs;
+      const int64_t waves = (total + conc - 1) / conc;
+      const double per_key_ns = (0.45 * G + 0.35) * (gd ? 1.15 : 1.0);
+      const double cost = double(waves) * (per_key_ns * double(R) + 6000.0);
+      if (!found || cost < best) {
+        best = cost;
+        found = true;
+        p.grid = int(total);
+        p.cluster = cs;
+        p.keys_per_cta = R;
+        p.list_cap = list_cap;
+        p.stages = stages;
+        p.smem = smem;
+        p.waves = int(waves);
+        p.l2_bytes = 0;
+        p.dist_global = gd != 0;
+      }
     }
   }
   return found && p.grid > 0 && int64_t(p.grid) == U * p.cluster && U * p.cluster < (1ll << 31);
@@ -1148,10 +1163,10 @@ namespace {
 struct PlanKey {
   int dev, B, Hq, Hkv, k, page_shift;
   int64_t L;
-  bool shared;
+  bool shared, allow_gd;
   bool operator<(const PlanKey& o) const {
-    return std::tie(dev, B, Hq, Hkv, k, page_shift, L, shared) <
-           std::tie(o.dev, o.B, o.Hq, o.Hkv, o.k, o.page_shift, o.L, o.shared);
+    return std::tie(dev, B, Hq, Hkv, k, page_shift, L, shared, allow_gd) <
+           std::tie(o.dev, o.B, o.Hq, o.Hkv, o.k, o.page_shift, o.L, o.shared, o.allow_gd);
   }
 };
 std::mutex g_plan_mutex;
@@ -1160,21 +1175,22 @@ constexpr size_t kMaxPlans = 4096;
 }  // namespace
 
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
-                                    int page_shift, Plan& p) {
+                                    int page_shift, Plan& p, bool allow_gd) {
   int dev = 0;
   const int sms = current_device_sms(&dev);
   if (sms <= 0) {
     // no device visible: plan for a 148-SM part with the sm_100 shared-memory cap
-    return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, 148, 232448, false, p);
+    return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, 148, 232448, false,
+                            p);
   }
-  const PlanKey key{dev, B, Hq, Hkv, k, page_shift, L, shared};
+  const PlanKey key{dev, B, Hq, Hkv, k, page_shift, L, shared, allow_gd};
   std::lock_guard<std::mutex> lock(g_plan_mutex);
   const auto it = g_plans.find(key);
   if (it != g_plans.end()) {
     p = it->second.second;
     return it->second.first;
   }
-  const bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, sms,
+  const bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, sms,
                                    max_smem_optin(dev), true, p);
   int l2 = 0;
   if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
@@ -1197,8 +1213,17 @@ size_t cp_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k, bool shared)
   return 256 + size_t(p.grid) * cp_scratch_per_cta(shared ? 1 : G, BS, int(p.keys_per_cta));
 }
 
-// The decode workspace only carries the device error word (bounded copy waits).
-size_t decode_workspace_bytes(int, int, int, int64_t, int) { return 256; }
+// The decode workspace carries the device error word (bounded copy waits) and, when
+// the plan keeps distances outside shared memory (per-head selection over long CTA
+// ranges), every CTA's distances.
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k) {
+  Plan p;
+  if (Hkv <= 0 || Hq % Hkv ||
+      !decode_plan_for_current_device(B, Hq, Hkv, L, k, false, -1, p, true))
+    return 256;
+  if (!p.dist_global) return 256;
+  return 256 + size_t(p.grid) * (Hq / Hkv) * dist_stride(int(p.keys_per_cta)) * 2;
+}
 size_t decode_workspace_error_offset() { return 8; }
 
 template <int G, bool SH, int MD, typename T>
@@ -1281,7 +1306,14 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
   a.cp_partial = cpa ? cpa->partial_out : nullptr;
   if (cpa) a.idx_stride = int(std::min<int64_t>(kk, cpa->L_total));
   const int mode = cpa != nullptr ? kModeCP
-                   : lay.block_table != nullptr ? kModePaged : kModeContiguous;
+                   : lay.block_table != nullptr ? kModePaged
+                   : p.dist_global ? kModeContigGD : kModeContiguous;
+  if (mode == kModeContigGD) {   // planned for per-head selection only
+    if (shared) return cudaErrorInvalidValue;
+    a.dist_scratch = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + 256);
+    return launch_dt<false, kModeContigGD>(dt, G, a, p, stream);
+  }
+  a.dist_scratch = nullptr;
   if (shared) {
     return mode == kModeCP      ? launch_dt<true, kModeCP>(dt, G, a, p, stream)
            : mode == kModePaged ? launch_dt<true, kModePaged>(dt, G, a, p, stream)

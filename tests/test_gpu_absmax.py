@@ -94,6 +94,7 @@ def _query_alternatives(qv, ratio, cap=16):
     (1, {}, 64),
     (2, dict(L=3001), 128),
     (2, dict(L=2000, Hq=16, Hkv=2), 256),
+    (2, dict(L=1500, Hq=8, Hkv=8, B=2), 100),      # MHA, batch 2
 ])
 def test_decode_absmax_matches_oracle(cfg, over, k, shared):
     w = WORKLOADS[cfg].scaled(**over)

@@ -54,6 +54,8 @@ def _run_ranks(inp, codes, cuts, k, shared):
     (2, dict(L=3000, B=2), [0, 1200, 3000], 200, True),          # shared selection
     (1, {}, [0, 512, 1024], 64, False),                          # fp32, single head
     (2, dict(L=1000, Hq=4, Hkv=2), [0, 990, 1000], 600, False),  # a tiny slice, big budget
+    (2, dict(L=2500, Hq=16, Hkv=2), [0, 500, 1000, 1500, 2000, 2500], 128, True),  # 5 ranks
+    (2, dict(L=1201, Hq=8, Hkv=2), [0, 1, 1200, 1201], 64, False),   # one-position ranks
 ])
 def test_context_parallel_matches_oracle_and_single_gpu(cfg, over, cuts, k, shared):
     w = WORKLOADS[cfg].scaled(**over)

@@ -40,6 +40,7 @@ def _oracle_idx(qc, kc, lens, k, shared):
     (2, 32, 8, 2048, [2048, 1500], 4096, 64),        # one page holds a whole sequence
     (2, 16, 2, 9000, [8191, 9000], 512, 700),        # G = 8, chunk-sized pages
     (5, 4, 2, 700, [700, 13, 300, 699, 2], 32, 1000),  # budget above every length
+    (3, 16, 2, 3000, [1, 2999, 3000], 1, 77),        # G = 8, one-token pages, length 1
 ])
 def test_select_paged_random_codes(B, Hq, Hkv, Lmax, lens, page, k, shared):
     rng = np.random.default_rng(B * 97 + Lmax + page)
@@ -110,7 +111,7 @@ def _run_decode(inp, kc, lens, k, page, shared, paged=True):
     idx = torch.full((B, rows, min(k, Lmax)), -7, dtype=torch.int32, device="cuda")
     if paged:
         pc = make_block_table(lens, Lmax, page, seed=Lmax * 3 + page)
-        big = 1e4 if inp.k_cache.dtype == torch.float32 else 1e4
+        big = 1e4                      # spare pages: values that would wreck the output
         kp = upload(scatter_to_pages(inp.k_cache, pc, fill=big))
         vp = upload(scatter_to_pages(inp.v_cache, pc, fill=big))
         cp = upload(scatter_to_pages(torch.from_numpy(kc), pc, fill=0))

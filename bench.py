@@ -174,8 +174,11 @@ def run_ours(args, rank, world, local):
     if absmax and (args.paged or w.append):
         raise SystemExit("--thresholds absmax is measured on contiguous caches without append")
     layer_sets = []
+    planted = None   # layer 0's planted key positions [B, Hq, n] (planted workloads)
     for layer in range(w.layers):
         inp = generate(w, dev, layer=layer)
+        if layer == 0 and inp.planted is not None:
+            planted = inp.planted.cpu()
         codes = torch.empty(inp.k_cache.shape[:-1] + (32,), dtype=torch.uint8, device=dev)
         if absmax:
             ad.encode_keys_absmax(inp.k_cache, codes, 0, L, ratio)
@@ -293,10 +296,17 @@ def run_ours(args, rank, world, local):
         print(f"# graph capture failed ({e}); eager launches", file=sys.stderr)
     stream.synchronize()
 
+    # an event after every full-size replay as well: the median per-replay time
+    rep_events = []
+
     def timed_region():
         if use_graph:
             for _ in range(K // chunk):
                 graphs[0][1].replay()
+                if len(rep_events) < 4096:
+                    ev = torch.cuda.Event(enable_timing=True)
+                    ev.record(stream)
+                    rep_events.append(ev)
             if K % chunk:
                 graphs[-1][1].replay()
         else:
@@ -329,6 +339,9 @@ def run_ours(args, rank, world, local):
         torch.distributed.barrier()
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1)
+    marks = [e0] + rep_events
+    med_us = (statistics.median(a.elapsed_time(b) for a, b in zip(marks, marks[1:])) * 1e3 / chunk
+              if rep_events else None)
     ad.check_workspace(ws, stream)
     del graphs
 
@@ -387,8 +400,27 @@ def run_ours(args, rank, world, local):
     stream.synchronize()
     ms_e2e = f0.elapsed_time(f1)
 
+    # recall of the planted keys: one more step on layer 0 with its selections read back
+    recall = None
+    if planted is not None and not cpW and pc is None:
+        idx = torch.empty((w.B, w.Hkv if shared else w.Hq, min(k, L)), dtype=torch.int32,
+                          device=dev)
+        q, kc, vc, cd = sets[0][0]
+        with torch.cuda.stream(stream):
+            if absmax:
+                ad.decode_step_absmax(q, kc, vc, cd, L, k, ratio, ws, shared=shared, out=out,
+                                      idx_out=idx, stream=stream)
+            else:
+                decode(q, kc, vc, cd, L, k, t, ws, out=out, idx_out=idx, stream=stream)
+        stream.synchronize()
+        sel = idx.cpu().long()
+        hits = [torch.isin(planted[b, h], sel[b, h // w.G if shared else h]).double().mean()
+                for b in range(w.B) for h in range(w.Hq)]
+        recall = round(float(torch.stack(hits).mean()), 4)
+
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
     return dict(w=w, k=k, ms=ms, ms_e2e=ms_e2e, K=K, K2=K2, R=R, step_bytes=step_bytes,
+                us_median=med_us, recall=recall,
                 clocks=clocks, plan=plan, use_graph=use_graph,
                 launches=K * launches_per_step,
                 h2d=q_host.numel() * q_host.element_size(),
@@ -406,28 +438,113 @@ def oracle_inputs(w, seed_device="cpu"):
     return inp.t, q, K, V, oracle
 
 
-def cpu_baseline(w, k, budget_s=12.0, shared=False, absmax=False):
-    """The oracle's full decode step (all heads) on the host, repeated for about
-    budget_s seconds: effective GB/s over the same algorithmic bytes."""
-    t, q, K, V, oracle = oracle_inputs(w)
-    # key codes are cache state, built before timing; the query encode is timed
-    kc = oracle.encode_absmax(K, 0.5) if absmax else oracle.encode(K, t)
-    fn = oracle.decode_step_shared if shared else oracle.decode_step
-    n = 0
-    t0 = time.perf_counter()
-    while True:
-        qc = oracle.encode_absmax(q, 0.5) if absmax else None
-        fn(q, K, V, k, t, key_codes=kc, query_codes=qc)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or n >= 50:
-            break
-    per_step = el / n
-    return {"value": w.algorithmic_bytes(k, shared) / per_step / 1e9, "unit": "GB/s",
-            "cores": 1,
-            "kind": "oracle",
-            "sample": f"{n} full decode steps of the same workload (all {w.B * w.Hq} heads), "
-                      f"{per_step * 1e3:.0f} ms each, numpy float64, single thread"}
+def cpu_baseline(w, k, budget_s=12.0, shared=False, absmax=False, max_threads=16):
+    """The float64 oracle, as it stands, on the host cores over a bounded, seeded
+    sample of the workload.
+
+    A job is one (layer, sequence, kv head) unit, the kv head's G query heads run
+    through the oracle's own decode step on that unit's slice.  Key codes are cache
+    state and are built before timing; the query encode is timed.  Jobs are drawn in
+    a seeded order (two layers sampled for multi-layer workloads) and run on one
+    thread for about budget_s seconds; the step time is the mean job time times the
+    jobs in a step.  The same jobs are then run over a pool of
+    threads (threads over units; numpy releases the GIL in the array work), and, for
+    a workload with an append, the oracle's encode of the appended keys is timed on
+    its own."""
+    import concurrent.futures
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(7 + w.config)
+    G = w.G
+    layers = (sorted(int(x) for x in rng.choice(w.layers, size=min(w.layers, 2), replace=False))
+              if w.layers > 1 else [0])
+    jobs = [(layer, b, kv) for layer in layers for b in range(w.B) for kv in range(w.Hkv)]
+    order = rng.permutation(len(jobs))
+    jobs = [jobs[i] for i in order]
+    jobs_per_step = w.layers * w.B * w.Hkv
+    step_bytes = w.algorithmic_bytes(k, shared) * w.layers
+    inputs = {}
+    cache = {}
+
+    def layer_inputs(layer):
+        # the sampled layers (at most two) stay in host memory
+        if layer not in inputs:
+            inputs[layer] = generate(w, "cpu", layer=layer)
+        return inputs[layer]
+
+    def prepared(job, keep=1):
+        """(q slice, K, V, key codes) of a job, float64; keeps `keep` jobs' rows."""
+        layer, b, kv = job
+        if job not in cache:
+            while len(cache) >= keep:
+                cache.pop(next(iter(cache)))
+            inp = layer_inputs(layer)
+            K = inp.k_cache[b:b + 1, kv:kv + 1].double().numpy()
+            V = inp.v_cache[b:b + 1, kv:kv + 1].double().numpy()
+            kc = oracle.encode_absmax(K, 0.5) if absmax else oracle.encode(K, w.t)
+            cache[job] = (inp.q[b:b + 1, kv * G:(kv + 1) * G].double().numpy(), K, V, kc)
+        return cache[job]
+
+    def run(qs, K, V, kc):
+        qc = oracle.encode_absmax(qs, 0.5) if absmax else None
+        fn = oracle.decode_step_shared if shared else oracle.decode_step
+        fn(qs, K, V, k, w.t, key_codes=kc, query_codes=qc)
+
+    # one thread
+    times = []
+    i = 0
+    wall0 = time.perf_counter()
+    while sum(times) < budget_s and (i < len(jobs) or time.perf_counter() - wall0 < 3 * budget_s):
+        args_ = prepared(jobs[i % len(jobs)])
+        t0 = time.perf_counter()
+        run(*args_)
+        times.append(time.perf_counter() - t0)
+        i += 1
+    per_job = sum(times) / len(times)
+    per_step = per_job * jobs_per_step
+    whole = len(times) >= jobs_per_step and w.layers == 1
+    res = {"value": round(step_bytes / per_step / 1e9, 6), "unit": "GB/s", "cores": 1,
+           "kind": "oracle",
+           "sample": (f"{len(times)} oracle decode jobs (one kv head's {G} query heads each, "
+                      "seeded order"
+                      + (f", layers {layers}" if w.layers > 1 else "")
+                      + f"), {per_job * 1e3:.1f} ms each; step time = mean x {jobs_per_step} "
+                      + ("jobs (every job of the step timed)" if whole else "jobs (scaled)")
+                      + "; numpy float64, one thread")}
+
+    # threads over units
+    nproc = os.cpu_count() or 1
+    T = max(1, min(nproc, max_threads, len(jobs)))
+    if T > 1:
+        # the jobs of the first T kv heads (host memory: T kv heads' float64 rows),
+        # cycled to about budget_s / 2 seconds of pool time
+        sub = jobs[:T]
+        cache.clear()
+        work = [prepared(j, keep=len(sub)) for j in sub]
+        reps = max(1, math.ceil(T * budget_s / 2 / max(per_job, 1e-6) / len(work)))
+        with concurrent.futures.ThreadPoolExecutor(T) as pool:
+            t0 = time.perf_counter()
+            list(pool.map(lambda a_: run(*a_), work * reps))
+            wall = time.perf_counter() - t0
+        n_thr = len(work) * reps
+        del work
+        per_step_thr = wall / n_thr * jobs_per_step
+        res["threads"] = {"value": round(step_bytes / per_step_thr / 1e9, 6), "unit": "GB/s",
+                          "cores": T, "nproc": nproc,
+                          "sample": f"{n_thr} jobs ({len(sub)} distinct) over {T} threads, "
+                                    f"{wall:.2f} s wall; step time = wall / jobs x "
+                                    f"{jobs_per_step}"}
+    cache.clear()
+
+    # the append's key encode, on its own
+    if w.append:
+        inp = layer_inputs(0)
+        Ka = inp.k_cache[:, :, w.L - w.append:w.L].double().numpy()
+        t0 = time.perf_counter()
+        oracle.encode(Ka, w.t)
+        res["append_encode_ms"] = round((time.perf_counter() - t0) * 1e3, 2)
+    inputs.clear()
+    return res
 
 
 def run_reference(args):
@@ -535,6 +652,8 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": round(r["ms"] / r["K"], 6),
         "us_per_step": round(per_step_s * 1e6, 3),
+        "us_per_step_median_replay": (round(r["us_median"], 3) if r["us_median"] is not None
+                                      else None),
         "pct_of_roofline": round(100 * gbs_rank / peak, 2),
         "higher_is_better": True,
         "scaling": "weak",
@@ -564,6 +683,8 @@ def main():
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
+    if r["recall"] is not None:
+        line["recall_planted_keys"] = r["recall"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, k, shared=args.shared,
                                             absmax=args.thresholds == "absmax")

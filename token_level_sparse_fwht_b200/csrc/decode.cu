@@ -417,26 +417,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   // ---- distance scan: one key per thread per chunk, G heads per key
   {
     constexpr int GR = G > 4 ? 4 : G;
+    // A thread reads its key's 32-byte code as two 16-byte halves, the second half
+    // first where swz = 1 (neighbouring lane quads then hit different banks), and
+    // scores the words in that order.  The distance is a sum over word pairs, so
+    // the query's words are taken in the same order instead: word i of the key
+    // pairs with query word (i + 4 swz) mod 8 of a[], and thermometer word j of b[]
+    // (built from a pair of code words) with (j + 2 swz) mod 4.
+    const int swz = (tid >> 2) & 1;
     Therm qreg[GR];
+    // query thermometer words of head g in this thread's word order
+    const auto load_q = [&](int g, Therm& qt) {
+      const uint4* s = reinterpret_cast<const uint4*>(qth + g * 12);
+      const uint4 lo = s[swz], hi = s[swz ^ 1];
+      qt.a[0] = lo.x; qt.a[1] = lo.y; qt.a[2] = lo.z; qt.a[3] = lo.w;
+      qt.a[4] = hi.x; qt.a[5] = hi.y; qt.a[6] = hi.z; qt.a[7] = hi.w;
+      const uint2* s2 = reinterpret_cast<const uint2*>(qth + g * 12 + 8);
+      const uint2 b0 = s2[swz], b1 = s2[swz ^ 1];
+      qt.b[0] = b0.x; qt.b[1] = b0.y; qt.b[2] = b1.x; qt.b[3] = b1.y;
+    };
     if constexpr (G <= 4) {
 #pragma unroll
-      for (int g = 0; g < GR; ++g) {
-        const uint32_t* s = qth + g * 12;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qreg[g].a[i] = s[i];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) qreg[g].b[i] = s[8 + i];
-      }
+      for (int g = 0; g < GR; ++g) load_q(g, qreg[g]);
     }
-    const int swz = (tid >> 2) & 1;   // conflict-free 2 x 16 B reads of a 32 B code
     const uint32_t one = uint32_t(a.keys_per_cta > 0);   // 1, opaque to the compiler
     // the thermometer words of this thread's key in ring slot `sl`
     const auto load_key = [&](int sl, Therm& kt) {
       const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t(sl) * kChunk + tid) *
                                                         kCodeBytes);
       const uint4 xa = src[swz], xb = src[swz ^ 1];
-      const uint4 x0 = swz ? xb : xa, x1 = swz ? xa : xb;
-      const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const uint32_t wd[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
       make_therm(wd, kt, one);
     };
     // distances of NK keys (positions r[]; side effects only where valid[]), with the
@@ -451,13 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       for (int g0 = 0; g0 < G; g0 += GR) {
         if constexpr (G > 4) {
 #pragma unroll
-          for (int g = 0; g < GR; ++g) {
-            const uint4* s = reinterpret_cast<const uint4*>(qth + (g0 + g) * 12);
-            const uint4 p0v = s[0], p1v = s[1], p2v = s[2];
-            qreg[g].a[0] = p0v.x; qreg[g].a[1] = p0v.y; qreg[g].a[2] = p0v.z; qreg[g].a[3] = p0v.w;
-            qreg[g].a[4] = p1v.x; qreg[g].a[5] = p1v.y; qreg[g].a[6] = p1v.z; qreg[g].a[7] = p1v.w;
-            qreg[g].b[0] = p2v.x; qreg[g].b[1] = p2v.y; qreg[g].b[2] = p2v.z; qreg[g].b[3] = p2v.w;
-          }
+          for (int g = 0; g < GR; ++g) load_q(g0 + g, qreg[g]);
         }
 #pragma unroll
         for (int g = 0; g < GR; ++g) {
@@ -532,13 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         for (int g0 = 0; g0 < G; g0 += GR) {
           if constexpr (G > 4) {
 #pragma unroll
-            for (int g = 0; g < GR; ++g) {
-              const uint4* s = reinterpret_cast<const uint4*>(qth + (g0 + g) * 12);
-              const uint4 p0v = s[0], p1v = s[1], p2v = s[2];
-              qreg[g].a[0] = p0v.x; qreg[g].a[1] = p0v.y; qreg[g].a[2] = p0v.z; qreg[g].a[3] = p0v.w;
-              qreg[g].a[4] = p1v.x; qreg[g].a[5] = p1v.y; qreg[g].a[6] = p1v.z; qreg[g].a[7] = p1v.w;
-              qreg[g].b[0] = p2v.x; qreg[g].b[1] = p2v.y; qreg[g].b[2] = p2v.z; qreg[g].b[3] = p2v.w;
-            }
+            for (int g = 0; g < GR; ++g) load_q(g0 + g, qreg[g]);
           }
 #pragma unroll
           for (int g = 0; g < GR; ++g) {

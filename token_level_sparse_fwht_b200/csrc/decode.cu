@@ -181,14 +181,16 @@ __device__ __forceinline__ uint32_t lane_sign_bits(uint32_t w0, uint32_t w1) {
 }
 
 // Exclusive prefix over the block (thread order) of G counters per thread, and the
-// block totals, with one barrier: warp totals go to shared memory and every thread
-// adds up the totals of the warps before it.  `scan` holds two buffers of
-// kWarps x G words used alternately (by `parity`), so a call never overwrites
-// totals that a slower warp may still be reading from the previous call.
+// block totals, with one barrier: warp totals go to shared memory, then in every warp
+// lanes 0..kWarps-1 take one total each and a shuffle scan over them gives each
+// warp its offset and the block total.  `scan` holds two buffers of kWarps x G
+// words used alternately (by `parity`), so a call never overwrites totals that a
+// slower warp may still be reading from the previous call.
 template <int G>
 __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t (&total)[G],
                                                      uint32_t* scan, int parity, int lane,
                                                      int warp) {
+  static_assert(kWarps <= 32, "one warp total per lane");
   uint32_t* buf = scan + parity * kWarps * G;
   uint32_t inc[G];
 #pragma unroll
@@ -203,22 +205,18 @@ __device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t 
     if (lane == 31) buf[warp * G + g] = x;
   }
   __syncthreads();
-  uint32_t before[G], tot[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) before[g] = tot[g] = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const uint32_t x = buf[w * G + g];
-      tot[g] += x;
-      before[g] += w < warp ? x : 0u;
-    }
-  }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    v[g] = before[g] + inc[g] - v[g];
-    total[g] = tot[g];
+    uint32_t x = lane < kWarps ? buf[lane * G + g] : 0u;
+#pragma unroll
+    for (int o = 1; o < kWarps; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    // x: inclusive prefix of the warp totals (lane w: warps 0..w)
+    const uint32_t upto = __shfl_sync(0xffffffffu, x, (warp + 31) & 31);
+    total[g] = __shfl_sync(0xffffffffu, x, kWarps - 1);
+    v[g] = (warp > 0 ? upto : 0u) + inc[g] - v[g];
   }
 }
 

@@ -218,11 +218,13 @@ __device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane
   v[0] = a0 + a2; v[1] = a1 + a3; v[2] = a0 - a2; v[3] = a1 - a3;
 #pragma unroll
   for (int s = 1; s < 32; s <<= 1) {
-    const bool upper = (lane & s) != 0;
+    // lower lane of the pair: v + o; upper: o - v.  One fma with a +-1 factor (the
+    // product is exact, so this rounds exactly like the add or subtract)
+    const float sg = (lane & s) ? -1.0f : 1.0f;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const float o = __shfl_xor_sync(0xffffffffu, v[r], s);
-      v[r] = upper ? (o - v[r]) : (v[r] + o);
+      v[r] = fmaf(v[r], sg, o);
     }
   }
   const float inv_sqrt_d = 0.088388347648318440550f;   // 1 / sqrt(128)

@@ -63,6 +63,140 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ 
   }
 }
 
+// Tensor-core encoder for bf16 vectors with a fixed threshold: a warp transforms 16
+// vectors at a time.  In natural (Sylvester) order H_128 = H_8 (x) H_16: for
+// i = 16a + b and k = 16c + d, (-1)^popc(i & k) = (-1)^popc(a & c) (-1)^popc(b & d).
+// So each 16-dimension block c of the 16 vectors is multiplied by H_16 with
+// mma.m16n8k16 (bf16 x +-1 products are exact; fp32 accumulation), and the 8 blocks
+// are then butterflied in registers (H_8).  The MMA's k order inside a block is
+// permuted so that a lane's A registers hold 4 consecutive dimensions (one 8-byte
+// load per row and block): k = 2q, 2q+1 -> dimensions 4q, 4q+1 and k = 2q+8, 2q+9 ->
+// 4q+2, 4q+3 (q = lane % 4); B = H_16 takes its rows in the same order.  Codes are
+// compared against t sqrt(128) on the unscaled sums.
+constexpr int kMmaVecs = 16;
+
+// bf16 bits of H_16[d0][n] (low half) and H_16[d1][n] (high half): +-1.0
+__device__ __forceinline__ uint32_t h16_pair(int d0, int d1, int n) {
+  const uint32_t lo = (__popc(d0 & n) & 1) ? 0xBF80u : 0x3F80u;
+  const uint32_t hi = (__popc(d1 & n) & 1) ? 0xBF80u : 0x3F80u;
+  return lo | (hi << 16);
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t code_of(float y, float tt) {
+  return uint32_t(y >= -tt) + uint32_t(y >= 0.0f) + uint32_t(y >= tt);
+}
+
+// Same vector and row mapping as encode_rows_kernel; run is a multiple of 16.
+__global__ void __launch_bounds__(256) encode_rows_mma_kernel(
+    const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst, int64_t nvec, int64_t per,
+    int64_t stride, int64_t off, int64_t run, float t, const int32_t* __restrict__ ids,
+    int64_t id_limit) {
+  const int lane = threadIdx.x & 31;
+  const int gid = lane >> 2, q = lane & 3;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  int64_t v = warp * run;
+  const int64_t vend = min(nvec, v + run);
+  if (v >= vend) return;
+  // H_16 fragments: n-tile nt holds outputs 8 nt .. 8 nt + 7 (column n = 8 nt + gid)
+  uint32_t bfr[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    bfr[nt][0] = h16_pair(4 * q, 4 * q + 1, 8 * nt + gid);
+    bfr[nt][1] = h16_pair(4 * q + 2, 4 * q + 3, 8 * nt + gid);
+  }
+  const float tt = t * 11.313708498984761f;   // sqrt(128)
+  for (; v < vend; v += kMmaVecs) {
+    // this lane's two rows: vectors v + gid (h = 0) and v + gid + 8 (h = 1)
+    int64_t row[2];
+    bool ok[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t vv = v + gid + 8 * h;
+      ok[h] = vv < vend;
+      int64_t g = 0, pos = 0;
+      if (ok[h]) {
+        g = vv / per;
+        pos = vv - g * per;
+        if (ids != nullptr) {
+          g = ids[g];
+          ok[h] = g >= 0 && g < id_limit;
+        }
+      }
+      row[h] = g * stride + off + pos;
+    }
+    uint2 x[2][8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint2* rp = reinterpret_cast<const uint2*>(src + row[h] * kD) + q;
+#pragma unroll
+      for (int a = 0; a < 8; ++a) x[h][a] = ok[h] ? __ldg(rp + 4 * a) : make_uint2(0u, 0u);
+    }
+    // z[c][nt][.]: block c times H_16; rows (gid, gid + 8) x columns 8 nt + 2 q + {0, 1}
+    float z[8][2][4];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        z[c][nt][0] = z[c][nt][1] = z[c][nt][2] = z[c][nt][3] = 0.0f;
+        mma_bf16_16816(z[c][nt], x[0][c].x, x[1][c].x, x[0][c].y, x[1][c].y, bfr[nt][0],
+                       bfr[nt][1]);
+      }
+    }
+    // H_8 over the block index
+#pragma unroll
+    for (int s = 1; s < 8; s <<= 1) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c & s) continue;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = z[c][nt][e], p1 = z[c | s][nt][e];
+            z[c][nt][e] = p0 + p1;
+            z[c | s][nt][e] = p0 - p1;
+          }
+        }
+      }
+    }
+    // codes: output dimension 16 a + 8 nt + 2 q + e.  A lane's two coordinates form
+    // half a byte; the xor-1 partner holds the other half, the xor-2 pair the next
+    // byte, so after two shuffles lane q = 0 of each quad has its row's 32 bytes.
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t word[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        uint32_t half[2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint32_t nib = code_of(z[a][nt][2 * h], tt) | (code_of(z[a][nt][2 * h + 1], tt) << 2);
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+          const uint32_t byte = (q & 1) ? (other | (nib << 4)) : (nib | (other << 4));
+          const uint32_t next = __shfl_xor_sync(0xffffffffu, byte, 2);
+          half[nt] = (q & 2) ? (next | (byte << 8)) : (byte | (next << 8));
+        }
+        word[a] = half[0] | (half[1] << 16);
+      }
+      if (q == 0 && ok[h]) {
+        uint4* d = reinterpret_cast<uint4*>(dst + row[h] * kCodeBytes);
+        d[0] = make_uint4(word[0], word[1], word[2], word[3]);
+        d[1] = make_uint4(word[4], word[5], word[6], word[7]);
+      }
+    }
+  }
+}
+
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,
                                int64_t per, int64_t stride, int64_t off, float t,
                                cudaStream_t stream, const int32_t* ids, int64_t id_limit,
@@ -76,7 +210,18 @@ cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, i
   const int64_t run = (nvec + warps - 1) / warps;
   const int64_t used = (nvec + run - 1) / run;
   const int grid = static_cast<int>((used + 7) / 8);
-  if (dt == ADAMAS_BF16) {
+  if (dt == ADAMAS_BF16 && ratio == 0.0f && reinterpret_cast<uintptr_t>(dst) % 16 == 0 &&
+      reinterpret_cast<uintptr_t>(src) % 8 == 0) {
+    // 2 blocks of 8 warps per SM; each warp a run of whole 16-vector tiles
+    const int64_t mw_max = int64_t(sms > 0 ? sms : 148) * 16;
+    const int64_t tiles = (nvec + kMmaVecs - 1) / kMmaVecs;
+    const int64_t mw = tiles < mw_max ? tiles : mw_max;
+    const int64_t mrun = (tiles + mw - 1) / mw * kMmaVecs;
+    const int64_t mused = (nvec + mrun - 1) / mrun;
+    encode_rows_mma_kernel<<<static_cast<int>((mused + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, mrun, t, ids,
+        id_limit);
+  } else if (dt == ADAMAS_BF16) {
     encode_rows_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, run, t, ids,
         id_limit, ratio);

@@ -97,6 +97,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the grid launched before this
+// one in the stream has completed and its memory is visible (a no-op when there is no
+// such dependency); every kernel calls it before its first global-memory access.
+// pdl_trigger: let the next grid in the stream begin launching its blocks (they run
+// up to their own pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Bounded wait on an mbarrier phase; records kErrCopy and returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint32_t* err) {

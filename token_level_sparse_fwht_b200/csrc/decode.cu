@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   constexpr bool paged = MD == kModePaged;
   constexpr bool cp = MD == kModeCP;   // one rank's slice of a context-parallel step
   extern __shared__ __align__(128) uint8_t smem[];
+  pdl_wait();
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = a.cluster;
   const int rank = int(cluster.block_rank());
@@ -659,6 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   }
 
   cluster.sync();   // cumulative histograms complete; coarse counts delivered
+  pdl_trigger();    // the next grid's blocks may take the SMs this one leaves idle
 
   if constexpr (cp) {
     if (a.cp_phase == 1) {
@@ -1230,13 +1232,15 @@ static cudaError_t launch_g(const DecodeArgs& a, const Plan& p, cudaStream_t str
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = p.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_kernel<G, SH, MD, T>, a);
 }
 

@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ 
                                                           int64_t run, float t,
                                                           const int32_t* __restrict__ ids,
                                                           int64_t id_limit, float ratio) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   using R = Raw4<T>;
@@ -101,6 +103,8 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
     const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst, int64_t nvec, int64_t per,
     int64_t stride, int64_t off, int64_t run, float t, const int32_t* __restrict__ ids,
     int64_t id_limit) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int gid = lane >> 2, q = lane & 3;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -210,6 +214,14 @@ cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, i
   const int64_t run = (nvec + warps - 1) / warps;
   const int64_t used = (nvec + run - 1) / run;
   const int grid = static_cast<int>((used + 7) / 8);
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (dt == ADAMAS_BF16 && ratio == 0.0f && reinterpret_cast<uintptr_t>(dst) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(src) % 8 == 0) {
     // 2 blocks of 8 warps per SM; each warp a run of whole 16-vector tiles
@@ -218,19 +230,18 @@ cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, i
     const int64_t mw = tiles < mw_max ? tiles : mw_max;
     const int64_t mrun = (tiles + mw - 1) / mw * kMmaVecs;
     const int64_t mused = (nvec + mrun - 1) / mrun;
-    encode_rows_mma_kernel<<<static_cast<int>((mused + 7) / 8), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, mrun, t, ids,
-        id_limit);
-  } else if (dt == ADAMAS_BF16) {
-    encode_rows_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off, run, t, ids,
-        id_limit, ratio);
-  } else {
-    encode_rows_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(src), dst,
-                                                         nvec, per, stride, off, run, t, ids,
-                                                         id_limit, ratio);
+    cfg.gridDim = dim3(static_cast<unsigned>((mused + 7) / 8));
+    return cudaLaunchKernelEx(&cfg, encode_rows_mma_kernel,
+                              static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off,
+                              mrun, t, ids, id_limit);
   }
-  return cudaGetLastError();
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  if (dt == ADAMAS_BF16)
+    return cudaLaunchKernelEx(&cfg, encode_rows_kernel<__nv_bfloat16>,
+                              static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off,
+                              run, t, ids, id_limit, ratio);
+  return cudaLaunchKernelEx(&cfg, encode_rows_kernel<float>, static_cast<const float*>(src), dst,
+                            nvec, per, stride, off, run, t, ids, id_limit, ratio);
 }
 
 }  // namespace adamas

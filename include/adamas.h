@@ -15,6 +15,10 @@
  *    adamas_check_workspace, which says so), and keeps no per-call host state.
  *  - Every call is asynchronous on `stream`; argument checks run on the host
  *    before any launch, and a rejected call launches nothing.
+ *  - Stream order is kept.  The decode and key-encode kernels are launched with
+ *    programmatic dependent launch: their blocks may become resident while the
+ *    previous kernel in the stream is still running, but wait for its completion
+ *    (and for its memory) before they touch any buffer.
  *  - Layouts are contiguous, row-major:
  *        q        [B][Hq][d]           elements of `dt`
  *        k_cache  [B][Hkv][Lmax][d]    elements of `dt`   (original keys)

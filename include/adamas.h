@@ -80,6 +80,10 @@ int adamas_abi_version(void);
  * transform, bucketization, 2-bit compression of the keys).  Encodes positions
  * [pos0, pos0 + n_new) of every (batch, kv head) from k_cache into codes.
  * Reads n_new * B * Hkv * d elements, writes n_new * B * Hkv * d/4 bytes.
+ * The transform runs in fp32 (bf16 keys with a fixed t: on the tensor cores, as
+ * H_8 x H_16), so a coordinate within rounding distance of a threshold may land
+ * in either neighbouring bucket; the fused decode step encodes its queries with a
+ * differently ordered fp32 FWHT.
  */
 adamas_status adamas_encode_keys(const void* k_cache, adamas_dtype dt, int B, int Hkv, int d,
                                  int64_t Lmax, int64_t pos0, int64_t n_new, float t,
@@ -91,11 +95,15 @@ adamas_status adamas_encode_queries(const void* q, adamas_dtype dt, int B, int H
 
 /*
  * Workspace of adamas_decode_step and adamas_select_topk, in bytes; 0 if the
- * arguments are invalid or unsupported.  The decode kernel keeps all its
- * intermediate data on chip, so the workspace only holds the device error word
- * that a bounded wait sets when it gives up (see adamas_check_workspace).  Zero-fill
- * it once before first use (adamas_workspace_init); any number of calls, on any
- * stream, may share it.
+ * arguments are invalid or unsupported.  The first 256 bytes hold the device error
+ * word that a bounded wait sets when it gives up (see adamas_check_workspace).
+ * Where the launch plan keeps every CTA's distances on chip (the 32K layer, for
+ * one) that is all of it.  Plans for long contexts over many (batch, kv head) units
+ * keep the distances in workspace scratch instead: one u16 per key and query head,
+ * written and read back by the same launch (it stays in L2).  Zero-fill the
+ * workspace once before first use (adamas_workspace_init); the scratch needs no
+ * initialisation.  Calls that run one after another on one stream may share a
+ * workspace; concurrent calls whose plans use scratch need one workspace each.
  */
 size_t adamas_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k);
 

@@ -18,7 +18,7 @@ Attention for Efficient Long-Context Inference", arXiv 2510.18413):
   three thresholds and strict "<" comparisons map a value to a bucket 0..3;
   section 3.1: the 2-bit codes are packed several to a machine word.
 
-Readings where the pages are silent or garbled (each one is listed in the design doc):
+Readings where the pages are silent or garbled:
 
 * H is the Sylvester matrix in natural order, H[i, j] = (-1)^popcount(i & j),
   scaled by 1/sqrt(d) so that it is orthonormal (the (HQ)(HK)^T identity of blog

@@ -1,6 +1,8 @@
 // Key and query encoders: orthonormal FWHT (d = 128), 2-bit buckets at
-// {-t, 0, +t}, 4 codes per byte.  One warp per vector, four vectors in flight per
-// warp (256 B read + 32 B written per bf16 key).
+// {-t, 0, +t}, 4 codes per byte (256 B read + 32 B written per bf16 key).  bf16
+// vectors with a fixed threshold go through the tensor cores, 16 vectors per warp;
+// fp32 vectors and per-vector (absmax) thresholds through a warp-shuffle FWHT, one
+// warp per vector with four in flight.
 //
 // Method: "Adamas: Hadamard Sparse Attention for Efficient Long-Context
 // Inference", v2 abstract (Hadamard transform, bucketization, 2-bit compression)

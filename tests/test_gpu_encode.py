@@ -77,3 +77,19 @@ def test_encode_full_append_workload():
     bad, frac, near = encoder_mismatch(codes[:, :, pos0:].cpu().numpy(), sub, inp.t)
     print(f"append encode: mismatch fraction {frac:.3g}, near-threshold fraction {near:.3g}")
     assert bad == 0 and frac < MAX_MISMATCH_FRACTION
+
+
+@pytest.mark.parametrize("n_new,pos0", [(1, 699), (3, 250), (17, 0)])
+def test_encode_short_appends(n_new, pos0):
+    """Appends shorter than a 16-key tile (one token per sequence per decode step is
+    the usual case): a tile then spans several (batch, kv head) rows."""
+    w = WORKLOADS[3].scaled(B=3, L=700)
+    inp = generate(w, "cpu")
+    k = inp.k_cache.cuda()
+    codes = torch.full(k.shape[:-1] + (32,), 0xAB, dtype=torch.uint8, device="cuda")
+    ad.encode_keys(k, codes, pos0, n_new, inp.t)
+    c = codes.cpu().numpy()
+    assert np.all(c[:, :, :pos0] == 0xAB) and np.all(c[:, :, pos0 + n_new:] == 0xAB)
+    bad, frac, _ = encoder_mismatch(c[:, :, pos0:pos0 + n_new],
+                                    inp.k_cache[:, :, pos0:pos0 + n_new], inp.t)
+    assert bad == 0 and frac < 1e-2      # few coordinates: one flip is 1/(B Hkv n 128)

@@ -90,3 +90,30 @@ def upload(x, device="cuda"):
     if isinstance(x, np.ndarray):
         x = torch.from_numpy(np.ascontiguousarray(x))
     return x.to(device).contiguous()
+
+
+def group_alternatives(qg: np.ndarray, t: float, cap: int = 64):
+    """Packed query codes [G, 32] the kernel may compute for one group qg [G, 128]:
+    every combination of the heads' admissible codes (at most `cap`)."""
+    per_head = [query_alternatives(qg[g], t) for g in range(qg.shape[0])]
+    for combo in itertools.islice(itertools.product(*per_head), cap):
+        yield np.stack(combo)
+
+
+def check_decode_unit_shared(gpu_idx, gpu_out, qg, Kg, Vg, kcg, k, t):
+    """One (batch, kv head) of a shared-selection step, given the group's queries qg
+    [G, 128], the unit's rows Kg, Vg [L, 128] and key codes kcg [L, 32]: the GPU's
+    selection must equal the oracle's for one admissible combination of the group's
+    query codes, and its outputs [G, 128] must be within ATOL_OUT of that selection's
+    attention.  Returns the max-abs error."""
+    errs = []
+    for qcg in group_alternatives(qg, t):
+        idx, out = oracle.decode_step_shared(qg[None], Kg[None, None], Vg[None, None], k, t,
+                                             key_codes=kcg[None, None], query_codes=qcg[None])
+        if not np.array_equal(np.asarray(gpu_idx, np.int64), idx[0, 0]):
+            continue
+        err = float(np.abs(np.asarray(gpu_out, np.float64) - out[0]).max())
+        errs.append(err)
+        if err <= ATOL_OUT:
+            return err
+    raise AssertionError(f"no admissible oracle selection matches: {errs}")

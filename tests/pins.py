@@ -10,6 +10,10 @@ What pins what:
   closed forms.
 * Codes: hand-written golden cases (tests/golden/bucket_cases.txt) for the strict
   "<" chain of blog section 2.2.
+* Threshold margin (which GPU encoder mismatches are forgiven): hand-worked rows
+  (tests/golden/margin_cases.txt, float32 rounding of t included) and the property
+  that moving y by less than its margin never changes its bucket, by slightly more
+  always can.
 * Packing: hand-worked bytes (tests/golden/pack_cases.txt).
 * Distance: the |a-b| table (tests/golden/manhattan_table.txt), a pure-Python brute
   force, and the t = 0 reduction to 3 x Hamming distance of sign bits (SimHash).
@@ -17,6 +21,10 @@ What pins what:
 * Attention: budget = L equals torch's dense scaled-dot-product attention; budget 1
   returns the V row.
 * GQA mapping and recall of planted keys on the seeded single-head workload.
+* decode_head (one query head, used to sample the big workloads and to enumerate the
+  admissible query codes): equal to decode_step's row for that head, with natural
+  and with explicitly given (different) key and query codes, and to a pure-Python
+  brute force of distance, selection and dense attention.
 * Shared selection: G = 1 reduction, pure-Python brute force, identical heads.
 * Per-sequence lengths: pure-Python brute force (empty, short and long sequences,
   -1 padding), invariance to cache slots past a length, full-length reduction.
@@ -117,6 +125,28 @@ def check_pack_golden():
 
 
 # --------------------------------------------------------------- distances
+def check_margin_golden():
+    """threshold_margin on hand-worked rows, float32(t) rounding included."""
+    for t, y, m in _golden("margin_cases.txt"):
+        got = float(ref.threshold_margin(np.array([float(y)]), float(t))[0])
+        assert abs(got - float(m)) <= 1e-15 + 1e-12 * float(m), (t, y, m, got)
+
+
+def check_margin_is_bucket_distance():
+    """Moving y by less than its margin keeps its bucket; by slightly more, one way
+    or the other changes it (bucketize is pinned by its own golden cases)."""
+    rng = np.random.default_rng(83)
+    for t in (0.0, 0.5, 1.01165):
+        y = rng.uniform(-3.5, 3.5, 4000)
+        m = ref.threshold_margin(y, t)
+        y, m = y[m > 1e-6], m[m > 1e-6]
+        c = ref.bucketize(y, t)
+        assert np.array_equal(ref.bucketize(y - 0.999 * m, t), c)
+        assert np.array_equal(ref.bucketize(y + 0.999 * m, t), c)
+        moved = (ref.bucketize(y - 1.001 * m, t) != c) | (ref.bucketize(y + 1.001 * m, t) != c)
+        assert moved.all()
+
+
 def check_manhattan_table():
     table = np.array([[int(x) for x in r] for r in _golden("manhattan_table.txt")])
     for a in range(4):
@@ -249,6 +279,39 @@ def check_planted_recall_single_head():
 
 
 # ---------------------------------------------------- shared GQA selection
+def check_decode_head_matches_step():
+    """decode_head(one head) = decode_step's row for that head, both with the codes it
+    encodes itself and with given key / query codes that differ from those; and equal
+    to a pure-Python brute force of the distances, the selection and the attention."""
+    rng = np.random.default_rng(89)
+    t, k = 0.5, 9
+    q = rng.standard_normal((1, 4, 128))
+    K = rng.standard_normal((1, 2, 60, 128))
+    V = rng.standard_normal((1, 2, 60, 128))
+    kc_alt = ref.encode(rng.standard_normal((1, 2, 60, 128)), t)
+    qc_alt = ref.encode(rng.standard_normal((1, 4, 128)), t)
+    i0, o0 = ref.decode_step(q, K, V, k, t)
+    i1, o1 = ref.decode_step(q, K, V, k, t, key_codes=kc_alt, query_codes=qc_alt)
+    differs = 0
+    for h in range(4):
+        kv = h // 2
+        sel, out, dist = ref.decode_head(q[0, h], K[0, kv], V[0, kv], k, t)
+        assert np.array_equal(sel, i0[0, h]) and np.allclose(out, o0[0, h], atol=1e-12)
+        sel1, out1, dist1 = ref.decode_head(q[0, h], K[0, kv], V[0, kv], k, t,
+                                            key_codes_rows=kc_alt[0, kv],
+                                            query_code=qc_alt[0, h])
+        assert np.array_equal(sel1, i1[0, h]) and np.allclose(out1, o1[0, h], atol=1e-12)
+        cq = ref.unpack_codes(qc_alt[0, h])
+        ck = ref.unpack_codes(kc_alt[0, kv])
+        brute = [sum(abs(int(cq[i]) - int(ck[j, i])) for i in range(128)) for j in range(60)]
+        assert [int(x) for x in dist1] == brute
+        want = _brute_select(brute, k)
+        assert list(sel1) == want
+        assert np.allclose(out1, _dense(q[0, h], K[0, kv, want], V[0, kv, want]), atol=1e-12)
+        differs += not np.array_equal(sel, sel1)
+    assert differs, "the substituted codes must change some selection"
+
+
 def check_shared_g1_is_per_head():
     """With one query head per kv head, shared selection IS per-head selection."""
     rng = np.random.default_rng(31)
@@ -478,6 +541,7 @@ ALL_CHECKS = [
     check_simhash_reduction, check_topk_bruteforce, check_topk_special,
     check_attention_dense, check_attention_budget1, check_decode_dense_limit,
     check_gqa_and_planted, check_planted_recall_single_head,
+    check_margin_golden, check_margin_is_bucket_distance, check_decode_head_matches_step,
     check_shared_g1_is_per_head, check_shared_bruteforce, check_shared_identical_heads,
     check_varlen_bruteforce, check_varlen_ignores_tail, check_varlen_uniform_is_decode_step,
     check_absmax_golden, check_bucket_per_vector_golden, check_absmax_reduces_to_fixed, check_absmax_extreme_coordinate,

@@ -14,7 +14,8 @@ import torch
 
 import oracle
 import token_level_sparse_fwht_b200 as ad
-from gpu_helpers import ATOL_OUT, f64, oracle_codes, query_alternatives, upload
+from gpu_helpers import (ATOL_OUT, check_decode_unit_shared as _check_unit, f64,
+                         oracle_codes, query_alternatives, upload)
 from workloads import WORKLOADS, generate
 
 pytestmark = pytest.mark.gpu
@@ -93,30 +94,6 @@ def test_select_shared_g1_equals_per_head():
     ws = ad.decode_workspace(B, Hq, Hkv, L, k)
     per_head = ad.select_topk(upload(qc), upload(kc), L, k, ws).cpu().numpy()
     assert np.array_equal(_select(qc, kc, L, k), per_head)
-
-
-def _group_alternatives(qg, t, cap=64):
-    """Packed query codes [G, 32] the kernel may compute for one group qg [G, 128]."""
-    per_head = [query_alternatives(qg[g], t) for g in range(qg.shape[0])]
-    for combo in itertools.islice(itertools.product(*per_head), cap):
-        yield np.stack(combo)
-
-
-def _check_unit(gpu_idx, gpu_out, qg, Kg, Vg, kcg, k, t):
-    """One (batch, kv head) of decode_step_shared, given the group's queries qg
-    [G, 128], the unit's first L rows Kg, Vg [L, 128] and codes kcg [L, 32]:
-    returns the max-abs error of the GPU output [G, 128]."""
-    errs = []
-    for qcg in _group_alternatives(qg, t):
-        idx, out = oracle.decode_step_shared(qg[None], Kg[None, None], Vg[None, None], k, t,
-                                             key_codes=kcg[None, None], query_codes=qcg[None])
-        if not np.array_equal(np.asarray(gpu_idx, np.int64), idx[0, 0]):
-            continue
-        err = float(np.abs(np.asarray(gpu_out, np.float64) - out[0]).max())
-        errs.append(err)
-        if err <= ATOL_OUT:
-            return err
-    raise AssertionError(f"no admissible oracle selection matches: {errs}")
 
 
 def _decode_shared(inp, kc, L, k):

@@ -13,7 +13,7 @@ _orig = {name: getattr(ref, name) for name in (
     "sylvester_hadamard", "hadamard_rotate", "bucketize", "pack_codes", "unpack_codes",
     "manhattan", "select_topk", "sparse_attention", "decode_step", "decode_step_shared",
     "decode_step_varlen", "absmax_thresholds", "bucketize_per_vector", "encode_absmax",
-    "decode_step_absmax")}
+    "decode_step_absmax", "threshold_margin", "decode_head")}
 
 
 def _h_or(n=128):                      # popcount(i | j) instead of i & j
@@ -168,6 +168,40 @@ def _decode_absmax_fixed_query(q, K, V, k, ratio=0.5, shared=False):
     return step(q, K, V, k, ratio, key_codes=_orig["encode_absmax"](K, ratio))
 
 
+def _margin_scaled(y, t):               # margin in unscaled units (x sqrt(d))
+    return _orig["threshold_margin"](y, t) * np.sqrt(128)
+
+
+def _margin_no_zero(y, t):              # the 0 threshold forgotten
+    y = np.asarray(y, np.float64)
+    tt = float(np.float32(t))
+    return np.minimum(np.abs(y + tt), np.abs(y - tt))
+
+
+def _margin_f64_t(y, t):                # t kept in float64, not the kernels' float32
+    y = np.asarray(y, np.float64)
+    t = float(t)
+    return np.minimum(np.minimum(np.abs(y + t), np.abs(y)), np.abs(y - t))
+
+
+def _head_ignores_query_code(q_vec, K_rows, V_rows, k, t, key_codes_rows=None,
+                             query_code=None):
+    return _orig["decode_head"](q_vec, K_rows, V_rows, k, t, key_codes_rows=key_codes_rows)
+
+
+def _head_ignores_key_codes(q_vec, K_rows, V_rows, k, t, key_codes_rows=None,
+                            query_code=None):
+    return _orig["decode_head"](q_vec, K_rows, V_rows, k, t, query_code=query_code)
+
+
+def _head_kv_swapped(q_vec, K_rows, V_rows, k, t, key_codes_rows=None, query_code=None):
+    # V rows used as keys in the attention (the codes still come from the keys)
+    if key_codes_rows is None:
+        key_codes_rows = ref.encode(K_rows, t)
+    return _orig["decode_head"](q_vec, V_rows, K_rows, k, t, key_codes_rows=key_codes_rows,
+                                query_code=query_code)
+
+
 MUTATIONS = {
     "hadamard_or": ("sylvester_hadamard", _h_or),
     "rotate_unscaled": ("hadamard_rotate", _rotate_unscaled),
@@ -191,6 +225,12 @@ MUTATIONS = {
     "absmax_inverse_ratio": ("absmax_thresholds", _absmax_inverse_ratio),
     "absmax_bucket_le": ("bucketize_per_vector", _per_vector_le),
     "absmax_fixed_query": ("decode_step_absmax", _decode_absmax_fixed_query),
+    "margin_scaled": ("threshold_margin", _margin_scaled),
+    "margin_no_zero_threshold": ("threshold_margin", _margin_no_zero),
+    "margin_float64_t": ("threshold_margin", _margin_f64_t),
+    "head_ignores_query_code": ("decode_head", _head_ignores_query_code),
+    "head_ignores_key_codes": ("decode_head", _head_ignores_key_codes),
+    "head_kv_swapped": ("decode_head", _head_kv_swapped),
 }
 
 

@@ -221,7 +221,7 @@ adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream
   if (cudaMemcpyAsync(&word, p, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return ADAMAS_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
-  if (word & (kErrBarrier | kErrCopy)) return ADAMAS_ERR_TIMEOUT;
+  if (word & kErrCopy) return ADAMAS_ERR_TIMEOUT;
   if (word & kErrInput) return ADAMAS_ERR_INVALID_ARG;
   return word ? ADAMAS_ERR_INTERNAL : ADAMAS_OK;
 }

@@ -16,8 +16,7 @@ constexpr int kBinStride = 388;         // padded histogram row
 constexpr int kPartStride = 132;        // m, l, 2 pad, acc[128] (floats)
 
 // error word bits (workspace header)
-constexpr uint32_t kErrBarrier = 1u;
-constexpr uint32_t kErrCopy = 2u;
+constexpr uint32_t kErrCopy = 2u;     // a bounded wait for a copy or a peer gave up
 constexpr uint32_t kErrSelect = 4u;   // top-k bookkeeping found no k-th distance
 constexpr uint32_t kErrInput = 8u;    // a device-resident length or page id out of range
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
@@ -121,49 +120,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void red_add_gpu(uint32_t* p, uint32_t v) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Grid-wide barrier for a cooperative launch (all CTAs co-resident).  Sense by
-// generation counter; the arrival counter returns to zero, so the workspace stays
-// reusable.  Bounded: gives up after kWaitLimitNs and records kErrBarrier.
-__device__ __forceinline__ void grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks,
-                                             uint32_t* err) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t g0 = ld_acquire_gpu(gen);
-    __threadfence();
-    const uint32_t arrived = atomicAdd(count, 1u) + 1u;
-    if (arrived == nblocks) {
-      atomicExch(count, 0u);
-      __threadfence();
-      st_release_gpu(gen, g0 + 1u);
-    } else {
-      const unsigned long long t0 = globaltimer_ns();
-      while (ld_acquire_gpu(gen) == g0) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          atomicOr(err, kErrBarrier);
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
-    __threadfence();
-  }
-  __syncthreads();
-}
-
 // L2 prefetch of one 128-element row (256 B bf16 / 512 B fp32), 128 B per line.
 template <typename T>
 __device__ __forceinline__ void prefetch_row_l2(const T* row) {
@@ -257,83 +213,74 @@ __device__ __forceinline__ uint32_t warp_fwht_code(float v[4], float t, int lane
 }
 
 // --------------------------------------------------------- code arithmetic
-// Thermometer form of a word of 16 packed codes: for code c = 2h + l the field
-// becomes (odd, even) = ([c >= 3], [c >= 1]).  Only c = 2 (binary 10) changes, to
-// 01: subtracting d = h & ~l at the even bit does it without borrows, as one
-// integer multiply-add w + d * neg1 (neg1 = 0xffffffff, held in a register the
-// compiler cannot fold) on the FMA pipe, leaving the logic pipe one op lighter.
-__device__ __forceinline__ uint32_t therm13(uint32_t w, uint32_t neg1) {
-  const uint32_t d = (w >> 1) & ~w & 0x55555555u;      // h & ~l, at the even bit
-  uint32_t r;
-  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(d), "r"(neg1), "r"(w));
-  return r;
-}
-// [c >= 2] of two words, the first at even bits, the second at odd bits.
-__device__ __forceinline__ uint32_t therm2(uint32_t w0, uint32_t w1) {
-  return ((w0 >> 1) & 0x55555555u) | (w1 & 0xaaaaaaaau);
-}
-
-// Thermometer words of one packed 32-byte code: 8 x therm13 + 4 x therm2.
-struct Therm {
-  uint32_t a[8];
-  uint32_t b[4];
+// Packed-pair form of one 32-byte code, for exact Manhattan distances with few
+// integer-logic operations.  A code word holds 16 fields c = 2h + l (l at the even
+// bit, h at the odd bit).  For 2-bit codes k, q:
+//   |k - q| = r0 + 2 r1,  r0 = l_k ^ l_q,
+//   r1 = [|k - q| >= 2] = (h_k ^ h_q) & (e_q | (l_k ^ h_q)),  e_q = [q in {0, 3}],
+// (all 16 cases check out: q = 0 gives h_k, q = 1 gives h_k l_k, q = 2 gives
+// ~h_k ~l_k, q = 3 gives ~h_k).  Words A = w[2j] and B = w[2j+1] are packed into three
+// words carrying one bit per coordinate of both, so that each of r0 and r1 costs one
+// or two LOP3 per 32 coordinates:
+//   p[j] = (A & EVEN) | ((B << 1) & ODD)   low bits: A's at even bits, B's at odd bits
+//   h[j] = (A & ODD) | ((B >> 1) & EVEN)   high bits: A's at odd bits, B's at even bits
+//   l[j] = ((A << 1) & ODD) | (B & EVEN)   low bits at the positions of h[j]
+// A key keeps p, h, l; a query keeps p, h and e = ~(h ^ l).  The two left shifts are
+// integer multiplies by an opaque 2 (`two`), so they run on the FMA pipe and leave
+// the integer-logic pipe, the scan's bottleneck, to the rest.
+struct PairWords {
+  uint32_t p[4], h[4], x[4];   // x: l for a key, e for a query
 };
 
-// `one` is 1 at run time, opaque to the compiler (see therm_dist_csa).
-__device__ __forceinline__ void make_therm(const uint32_t w[8], Therm& t, uint32_t one) {
-  const uint32_t neg1 = 0u - one;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t.a[i] = therm13(w[i], neg1);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) t.b[i] = therm2(w[2 * i], w[2 * i + 1]);
+__device__ __forceinline__ uint32_t mul_opaque(uint32_t a, uint32_t m) {
+  uint32_t r;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(m));
+  return r;
 }
 
-// Manhattan distance of two code vectors from their thermometer words:
-// |a - b| = [a>=1]^[b>=1] + [a>=2]^[b>=2] + [a>=3]^[b>=3] per coordinate.
-__device__ __forceinline__ uint32_t therm_dist(const Therm& k, const Therm& q) {
-  uint32_t s0 = 0, s1 = 0, s2 = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    s0 += __popc(k.a[2 * i] ^ q.a[2 * i]);
-    s1 += __popc(k.a[2 * i + 1] ^ q.a[2 * i + 1]);
-    s2 += __popc(k.b[i] ^ q.b[i]);
-  }
-  return s0 + s1 + s2;
-}
-
-// Same distance with two carry-save levels.  The 12 XOR words are added bitwise three
-// at a time (sum word = a^b^c, carry word = majority(a,b,c), both single LOP3s) into
-// four weight-1 and four weight-2 words; three of each are added again, leaving
-// weight-1 words O and o3, weight-2 words T1, T2 and t3, and one weight-4 word F:
-// 6 popcounts replace 12.  POPC issues at a quarter of the integer-logic rate on
-// sm_100, so this moves work from the popcount pipe to the logic pipe, where the
-// thermometer words' multiply-adds (therm13) made room.
-__device__ __forceinline__ uint32_t therm_dist_csa(const Therm& k, const Therm& q,
-                                                   uint32_t one) {
-  uint32_t x[12];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = k.a[i] ^ q.a[i];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) x[8 + i] = k.b[i] ^ q.b[i];
-  // The sums run as integer multiply-adds with a multiplier the compiler cannot
-  // fold (one == 1 at run time), which keeps them on the FMA pipe and leaves the
-  // integer-logic pipe, the scan's bottleneck, to the XOR / carry-save work.
-  uint32_t o[4], tw[4];
+// Key words of one packed code; `two` is 2 at run time, opaque to the compiler.
+__device__ __forceinline__ void make_pairs(const uint32_t w[8], PairWords& t, uint32_t two) {
+  constexpr uint32_t kEven = 0x55555555u;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t a = x[3 * j], b = x[3 * j + 1], c = x[3 * j + 2];
-    o[j] = a ^ b ^ c;
-    tw[j] = (a & b) | (c & (a | b));
+    const uint32_t A = w[2 * j], B = w[2 * j + 1];
+    const uint32_t A2 = mul_opaque(A, two), B2 = mul_opaque(B, two);
+    t.p[j] = (A & kEven) | (B2 & ~kEven);
+    t.h[j] = (A & ~kEven) | ((B >> 1) & kEven);
+    t.x[j] = (A2 & ~kEven) | (B & kEven);
   }
-  const uint32_t O = o[0] ^ o[1] ^ o[2];
-  const uint32_t T1 = (o[0] & o[1]) | (o[2] & (o[0] | o[1]));
-  const uint32_t T2 = tw[0] ^ tw[1] ^ tw[2];
-  const uint32_t F = (tw[0] & tw[1]) | (tw[2] & (tw[0] | tw[1]));
-  // sum = popc(O) + popc(o3) + 2 (popc(T1) + popc(T2) + popc(t3)) + 4 popc(F)
+}
+
+// Query words of one packed code: p, h and e = [q in {0, 3}] at the positions of h.
+__device__ __forceinline__ void make_query_pairs(const uint32_t w[8], PairWords& t) {
+  make_pairs(w, t, 2u);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) t.x[j] = ~(t.h[j] ^ t.x[j]);
+}
+
+// Manhattan distance of a key code (k) and a query code (q) in packed-pair form.
+// The four r0 words (weight 1) and four r1 words (weight 2) are added bitwise by one
+// carry-save level on three of each (sum word a^b^c, carry word majority(a,b,c), both
+// single LOP3s), which leaves weight-1 words O and u1[3], weight-2 words T1, T2 and
+// u2[3], and one weight-4 word F: 6 popcounts.  The popcount sums are integer
+// multiply-adds with the opaque multiplier `one` (1 at run time), on the FMA pipe.
+__device__ __forceinline__ uint32_t pair_dist(const PairWords& k, const PairWords& q,
+                                              uint32_t one) {
+  uint32_t u1[4], u2[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    u1[j] = k.p[j] ^ q.p[j];
+    u2[j] = (k.h[j] ^ q.h[j]) & (q.x[j] | (k.x[j] ^ q.h[j]));
+  }
+  const uint32_t O = u1[0] ^ u1[1] ^ u1[2];
+  const uint32_t T1 = (u1[0] & u1[1]) | (u1[2] & (u1[0] | u1[1]));
+  const uint32_t T2 = u2[0] ^ u2[1] ^ u2[2];
+  const uint32_t F = (u2[0] & u2[1]) | (u2[2] & (u2[0] | u2[1]));
+  // sum = popc(O) + popc(u1[3]) + 2 (popc(T1) + popc(T2) + popc(u2[3])) + 4 popc(F)
   uint32_t s1 = uint32_t(__popc(O)), s2 = uint32_t(__popc(T1));
-  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s1) : "r"(uint32_t(__popc(o[3]))), "r"(one));
+  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s1) : "r"(uint32_t(__popc(u1[3]))), "r"(one));
   asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s2) : "r"(uint32_t(__popc(T2))), "r"(one));
-  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s2) : "r"(uint32_t(__popc(tw[3]))), "r"(one));
+  asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(s2) : "r"(uint32_t(__popc(u2[3]))), "r"(one));
   uint32_t r;
   asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(s2), "r"(one + one), "r"(s1));
   asm("mad.lo.u32 %0, %1, %2, %0;" : "+r"(r) : "r"(uint32_t(__popc(F))), "r"(4u * one));

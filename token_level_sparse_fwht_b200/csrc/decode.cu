@@ -403,13 +403,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     uint32_t wd[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) wd[i] = wq[i];
-    Therm th;
-    make_therm(wd, th, uint32_t(a.keys_per_cta > 0));
+    PairWords th;
+    make_query_pairs(wd, th);
     uint32_t* dst = qth + tid * 12;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dst[i] = th.a[i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[8 + i] = th.b[i];
+    for (int j = 0; j < 4; ++j) {
+      dst[j] = th.p[j];
+      dst[4 + j] = th.h[j];
+      dst[8 + j] = th.x[j];
+    }
   }
   __syncthreads();
 
@@ -418,39 +420,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     constexpr int GR = G > 4 ? 4 : G;
     // A thread reads its key's 32-byte code as two 16-byte halves, the second half
     // first where swz = 1 (neighbouring lane quads then hit different banks), and
-    // scores the words in that order.  The distance is a sum over word pairs, so
-    // the query's words are taken in the same order instead: word i of the key
-    // pairs with query word (i + 4 swz) mod 8 of a[], and thermometer word j of b[]
-    // (built from a pair of code words) with (j + 2 swz) mod 4.
+    // scores the words in that order.  The distance is a sum over coordinates, so the
+    // query's packed-pair words are taken in the same order instead: key pair j (code
+    // words 2j, 2j+1 in load order) pairs with query pair (j + 2 swz) mod 4.
     const int swz = (tid >> 2) & 1;
-    Therm qreg[GR];
-    // query thermometer words of head g in this thread's word order
-    const auto load_q = [&](int g, Therm& qt) {
-      const uint4* s = reinterpret_cast<const uint4*>(qth + g * 12);
-      const uint4 lo = s[swz], hi = s[swz ^ 1];
-      qt.a[0] = lo.x; qt.a[1] = lo.y; qt.a[2] = lo.z; qt.a[3] = lo.w;
-      qt.a[4] = hi.x; qt.a[5] = hi.y; qt.a[6] = hi.z; qt.a[7] = hi.w;
-      const uint2* s2 = reinterpret_cast<const uint2*>(qth + g * 12 + 8);
-      const uint2 b0 = s2[swz], b1 = s2[swz ^ 1];
-      qt.b[0] = b0.x; qt.b[1] = b0.y; qt.b[2] = b1.x; qt.b[3] = b1.y;
+    PairWords qreg[GR];
+    // query words of head g in this thread's pair order
+    const auto load_q = [&](int g, PairWords& qt) {
+      const uint2* s = reinterpret_cast<const uint2*>(qth + g * 12);
+      const uint2 p0 = s[swz], p1 = s[swz ^ 1];
+      const uint2 h0 = s[2 + swz], h1 = s[2 + (swz ^ 1)];
+      const uint2 x0 = s[4 + swz], x1 = s[4 + (swz ^ 1)];
+      qt.p[0] = p0.x; qt.p[1] = p0.y; qt.p[2] = p1.x; qt.p[3] = p1.y;
+      qt.h[0] = h0.x; qt.h[1] = h0.y; qt.h[2] = h1.x; qt.h[3] = h1.y;
+      qt.x[0] = x0.x; qt.x[1] = x0.y; qt.x[2] = x1.x; qt.x[3] = x1.y;
     };
     if constexpr (G <= 4) {
 #pragma unroll
       for (int g = 0; g < GR; ++g) load_q(g, qreg[g]);
     }
     const uint32_t one = uint32_t(a.keys_per_cta > 0);   // 1, opaque to the compiler
-    // the thermometer words of this thread's key in ring slot `sl`
-    const auto load_key = [&](int sl, Therm& kt) {
+    const uint32_t two = one + one;
+    // the packed-pair words of this thread's key in ring slot `sl`
+    const auto load_key = [&](int sl, PairWords& kt) {
       const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t(sl) * kChunk + tid) *
                                                         kCodeBytes);
       const uint4 xa = src[swz], xb = src[swz ^ 1];
       const uint32_t wd[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-      make_therm(wd, kt, one);
+      make_pairs(wd, kt, two);
     };
     // distances of NK keys (positions r[]; side effects only where valid[]), with the
     // keys' work in one block so that their dependency chains interleave (the pair
     // loop below; the one-chunk loop keeps its own branch-guarded body)
-    const auto score_keys = [&](auto nk_tag, const Therm* kt, const int* r, const bool* valid) {
+    const auto score_keys = [&](auto nk_tag, const PairWords* kt, const int* r, const bool* valid) {
       constexpr int NK = decltype(nk_tag)::value;
       uint32_t dsum[NK];
 #pragma unroll
@@ -465,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         for (int g = 0; g < GR; ++g) {
 #pragma unroll
           for (int u = 0; u < NK; ++u) {
-            const uint32_t dd = therm_dist_csa(kt[u], qreg[g], one);
+            const uint32_t dd = pair_dist(kt[u], qreg[g], one);
             if constexpr (SH) {
               dsum[u] += dd;
             } else if (valid[u]) {
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           if (slot2 == S) { slot2 = 0; par2 ^= 1u; }
           mbar_wait_bounded(&mbar[slot], parity, a.err);
           mbar_wait_bounded(&mbar[slot2], par2, a.err);
-          Therm kt[2];
+          PairWords kt[2];
           load_key(slot, kt[0]);
           load_key(slot2, kt[1]);
           const int r[2] = {qi * kChunk + tid, (qi + 1) * kChunk + tid};
@@ -527,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
       const int r = qi * kChunk + tid;
       if (r < n) {
-        Therm kt;
+        PairWords kt;
         load_key(slot, kt);
         uint32_t dsum = 0;   // shared selection: sum of the G heads' distances
 #pragma unroll
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           }
 #pragma unroll
           for (int g = 0; g < GR; ++g) {
-            const uint32_t dd = therm_dist_csa(kt, qreg[g], one);
+            const uint32_t dd = pair_dist(kt, qreg[g], one);
             if constexpr (SH) {
               dsum += dd;
             } else {

@@ -1,13 +1,14 @@
 """Benchmark of the Adamas decode step on B200: µs per step and effective HBM GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--budget 128]
-                    [--shared] [--paged PAGE] [--thresholds fixed|absmax]
-                    [--impl ours|reference]
+                    [--shared] [--paged PAGE] [--thresholds fixed|absmax] [--cp W]
+                    [--policy auto|cluster|flat] [--no-per-config] [--impl ours|reference]
 
 Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32 query / 8 kv heads,
 d = 128, context 32768, bf16 K/V with 4 outlier channels, budget 128.  A "step" is
 one adamas_decode_step (query encode, distance scan, top-k, gather attention,
-combine: one thread-block-cluster kernel launch).  --shared times the variant with
+combine: one kernel launch).  The default line also carries `per_config`: every
+workload at the budgets it is quoted on, timed the same way.  --shared times the variant with
 one selection per kv head shared by its query heads (adamas_decode_step_shared);
 its algorithmic bytes count the selected K/V rows once per kv head.
 
@@ -15,8 +16,9 @@ Timing: inputs resident in HBM; R independent replicas of codes + K + V are
 rotated so the working set of consecutive steps exceeds 2x L2 (no cache reuse
 between steps); K steps are captured in CUDA graphs and timed with CUDA events on
 the launching stream, bracketed by barrier + synchronize; max over ranks.
-Multi-GPU: every rank runs its own replica set (weak scaling, no collective on the
-data path).  Rank 0 prints one JSON line.
+Multi-GPU: `--gpus N` starts N local ranks (torch.distributed.run) unless a launcher
+already set WORLD_SIZE; every rank runs its own replica set (weak scaling, no
+collective on the data path).  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -165,22 +167,29 @@ def smi_id(dev) -> str:
         return str(dev.index)
 
 
-def run_ours(args, rank, world, local):
+def measure(args, config, k, dev, world, per_config=False):
+    """One workload at one budget: data on the device, then the timed steps.
+
+    A step is one pass of the whole path over one batch: every layer's
+    adamas_decode_step (and, for the batch-8 workload, the adamas_encode_keys of the
+    appended tokens first).  K steps run in CUDA graphs on one stream, timed with
+    CUDA events and bracketed by barrier + synchronize; W graph replays come first.
+    Returns a dict of measurements (times are this rank's)."""
     import token_level_sparse_fwht_b200 as ad
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    w = WORKLOADS[args.config]
-    k = args.budget
+    w = WORKLOADS[config]
     L = w.L
     t = w.t
-    # one "set" = everything one decode step touches: per layer (q, K, V, codes)
-    absmax = args.thresholds == "absmax"
+    absmax = args.thresholds == "absmax" and not per_config
+    shared = args.shared and not per_config
+    paged = args.paged if not per_config else 0
+    cpW = args.cp if not per_config else 0
     ratio = 0.5
-    if absmax and (args.paged or w.append):
+    if absmax and (paged or w.append):
         raise SystemExit("--thresholds absmax is measured on contiguous caches without append")
     layer_sets = []
     planted = None   # layer 0's planted key positions [B, Hq, n] (planted workloads)
+    append_check = None
     for layer in range(w.layers):
         inp = generate(w, dev, layer=layer)
         if layer == 0 and inp.planted is not None:
@@ -190,22 +199,25 @@ def run_ours(args, rank, world, local):
             ad.encode_keys_absmax(inp.k_cache, codes, 0, L, ratio)
         else:
             ad.encode_keys(inp.k_cache, codes, 0, L, t)
+        if layer == 0 and w.append:
+            # the appended keys' codes against the oracle (outside the timed region)
+            append_check = (inp.k_cache[:, :, L - w.append:L].cpu(),
+                            codes[:, :, L - w.append:L].cpu())
         layer_sets.append((inp.q, inp.k_cache, inp.v_cache, codes))
         del inp
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     append = w.append
-    shared = args.shared
     decode = ad.decode_step_shared if shared else ad.decode_step
     step_bytes = w.algorithmic_bytes(k, shared) * w.layers
     if append:
         step_bytes += w.B * w.Hkv * append * (128 * w.elem_bytes + 32)
     pc = None
-    if args.paged:
+    if paged:
         # the same caches held in a page pool (shuffled pages, block table, lengths);
         # an append re-encodes the pages that hold the new positions
         from workloads.paging import make_block_table, scatter_to_pages
-        ps = args.paged
-        pc = make_block_table([L] * w.B, L, ps, seed=args.config, spare=0)
+        ps = paged
+        pc = make_block_table([L] * w.B, L, ps, seed=config, spare=0)
         bt = pc.block_table.to(dev)
         lens = pc.seq_lens.to(dev)
         app_ids = (pc.block_table[:, (L - append) // ps:(L + ps - 1) // ps].reshape(-1)
@@ -225,18 +237,16 @@ def run_ours(args, rank, world, local):
     out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
     plan = (ad.decode_plan_shared if shared else ad.decode_plan)(w.B, w.Hq, w.Hkv, L, k)
-    launches_per_step = w.layers * (2 if append else 1) * (1 if not args.cp else 3)
+    launches_per_step = w.layers * (2 if append else 1) * (1 if not cpW else 3)
 
-    cpW = args.cp
     if cpW:
         # one rank of a context-parallel step over W GPUs, on one GPU: this rank holds
         # the first L / W positions; both all-gathers are stood in for by a local copy
         # of this rank's own tensor into the gathered buffer (the NCCL transfer itself
         # is not timed)
-        if args.paged or absmax or append or w.layers > 1:
+        if paged or absmax or append or w.layers > 1:
             raise SystemExit("--cp is measured on one contiguous layer without append")
         Ls = L // cpW
-        rows = w.Hkv if shared else w.Hq
         hist_all = torch.empty((cpW,) + ad.cp_hist_shape(w.B, w.Hq, w.Hkv, shared),
                                dtype=torch.int32, device=dev)
         part_all = torch.empty((cpW, w.B, w.Hq, ad.PART_STRIDE), dtype=torch.float32,
@@ -302,34 +312,28 @@ def run_ours(args, rank, world, local):
         print(f"# graph capture failed ({e}); eager launches", file=sys.stderr)
     stream.synchronize()
 
-    # an event after every full-size replay as well: the median per-replay time
-    rep_events = []
-
-    def timed_region():
+    def replay_k():
+        """Exactly K steps."""
         if use_graph:
             for _ in range(K // chunk):
                 graphs[0][1].replay()
-                if len(rep_events) < 4096:
-                    ev = torch.cuda.Event(enable_timing=True)
-                    ev.record(stream)
-                    rep_events.append(ev)
             if K % chunk:
                 graphs[-1][1].replay()
         else:
             for i in range(K):
                 step(i, stream)
 
-    with torch.cuda.stream(stream):       # graph warm-up replays
-        for _ in range(max(1, args.warmup // max(1, chunk))):
+    sampler = ClockSampler(smi_id(dev)) if not per_config else None
+    if sampler:
+        sampler.start()
+    # W warm-up steps as graph replays, then the timed K steps right behind them (no
+    # idle gap: a GPU left idle drops its clocks)
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, math.ceil(args.warmup / max(1, chunk)))):
             if use_graph:
                 graphs[0][1].replay()
             else:
                 step(0, stream)
-    stream.synchronize()
-
-    sampler = ClockSampler(smi_id(dev))
-    sampler.start()
-    time.sleep(0.3)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -337,17 +341,26 @@ def run_ours(args, rank, world, local):
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        timed_region()
+        replay_k()
         e1.record(stream)
     stream.synchronize()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
     ms = e0.elapsed_time(e1)
-    marks = [e0] + rep_events
-    med_us = (statistics.median(a.elapsed_time(b) for a, b in zip(marks, marks[1:])) * 1e3 / chunk
-              if rep_events else None)
+    # the median over at least 10 more replays of the K steps (outside the timed region)
+    reps = []
+    with torch.cuda.stream(stream):
+        for _ in range(10 if K * launches_per_step <= 20000 else 3):
+            a_ = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            replay_k()
+            b_.record(stream)
+            reps.append((a_, b_))
+    stream.synchronize()
+    med_us = statistics.median(a_.elapsed_time(b_) for a_, b_ in reps) * 1e3 / K
+    clocks = sampler.stop() if sampler else None
     ad.check_workspace(ws, stream)
     del graphs
 
@@ -396,6 +409,7 @@ def run_ours(args, rank, world, local):
         for i in range(3):
             e2e_step(i)
     stream.synchronize()
+    # pipelined: K2 calls queued back to back between two events
     f0 = torch.cuda.Event(enable_timing=True)
     f1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -405,6 +419,16 @@ def run_ours(args, rank, world, local):
         f1.record(stream)
     stream.synchronize()
     ms_e2e = f0.elapsed_time(f1)
+    # synchronised: a serving loop that needs each step's output on the host before
+    # the next step (host clock from the call to the stream's completion)
+    sync_us = []
+    with torch.cuda.stream(stream):
+        for i in range(max(10, min(K2, 200))):
+            h0 = time.perf_counter()
+            e2e_step(i)
+            stream.synchronize()
+            sync_us.append((time.perf_counter() - h0) * 1e6)
+    sync_med = statistics.median(sync_us)
 
     # recall of the planted keys: one more step on layer 0 with its selections read back
     recall = None
@@ -424,13 +448,54 @@ def run_ours(args, rank, world, local):
                 for b in range(w.B) for h in range(w.Hq)]
         recall = round(float(torch.stack(hits).mean()), 4)
 
-    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+    del sets, layer_sets, calls, ws, out, q_host, out_host, q_dev, outs
+    torch.cuda.empty_cache()
+    ms, ms_e2e, med_us, sync_med = max_over_ranks([ms, ms_e2e, med_us, sync_med], world, dev)
+    flat = plan["cluster"] == 1 and plan["ctas"] > w.B * w.Hkv
     return dict(w=w, k=k, ms=ms, ms_e2e=ms_e2e, K=K, K2=K2, R=R, step_bytes=step_bytes,
-                us_median=med_us, recall=recall,
+                us_median=med_us, sync_us=sync_med, recall=recall, append_check=append_check,
                 clocks=clocks, plan=plan, use_graph=use_graph,
-                launches=K * launches_per_step,
-                h2d=q_host.numel() * q_host.element_size(),
-                d2h=out_host.numel() * out_host.element_size())
+                kernel="decode_flat_kernel" if flat else "decode_kernel",
+                launches=K * launches_per_step, h2d=h2d, d2h=d2h)
+
+
+# the bench line's per_config entries: every workload at the budgets it is quoted on
+PER_CONFIG = [(1, 64), (2, 64), (2, 128), (2, 256), (2, 1024), (3, 256), (3, 1024), (4, 128),
+              (4, 1024), (5, 1024)]
+
+
+def per_config_entry(r, peak):
+    w, k = r["w"], r["k"]
+    per_step_s = r["ms"] / 1e3 / r["K"]
+    gbs = aggregate_gbs(r["step_bytes"], per_step_s, 1)
+    e = {"workload": w.name, "k": k, "us_per_step": round(per_step_s * 1e6, 3),
+         "us_per_step_median_replay": round(r["us_median"], 3),
+         "gbs": round(gbs, 2), "frac": round(gbs / peak, 4),
+         "algorithmic_bytes_per_step": r["step_bytes"], "ctas": r["plan"]["ctas"],
+         "kernel": r["kernel"], "steps": r["K"],
+         "e2e_us_per_step": round(r["ms_e2e"] / 1e3 / r["K2"] * 1e6, 3),
+         "e2e_sync_us_per_step": round(r["sync_us"], 2)}
+    if r["recall"] is not None:
+        e["recall_planted_keys"] = r["recall"]
+    return e
+
+
+def cpu_append_baseline(w, keys, gpu_codes):
+    """CPU-baseline leg for a workload with an append: the float64 oracle encodes the
+    appended keys on one host core (timed), and the GPU encoder's codes of the same
+    keys are compared with it (the fraction of coordinates whose code differs; a
+    coordinate within rounding distance of a threshold may legitimately differ)."""
+    import oracle
+    kk = keys.double().numpy()
+    t0 = time.perf_counter()
+    want = oracle.encode(kk, w.t)
+    ms = (time.perf_counter() - t0) * 1e3
+    diff = oracle.unpack_codes(gpu_codes.numpy()) != oracle.unpack_codes(want)
+    return {"oracle_encode_ms": round(ms, 2), "cores": 1,
+            "gpu_code_mismatch_fraction": float(diff.mean()),
+            "sample": f"all {kk.shape[0] * kk.shape[1] * kk.shape[2]} appended keys of layer 0"}
 
 
 # --------------------------------------------------- float64 oracle on host
@@ -605,16 +670,58 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- main
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(n: int) -> int:
+    """`bench.py --gpus N` without a launcher: re-run this command under
+    torch.distributed.run with N local ranks (one GPU each) and return its exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def init_ranks(world, local):
+    import datetime
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+    torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return backend
+
+
+def launcher_check(world, local, rank):
+    """--launcher-check: the rank set-up and the max-over-ranks reduction alone (no
+    kernel runs; gloo when no GPU is visible)."""
+    backend = init_ranks(world, local) if world > 1 else "none"
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else None
+    got = max_over_ranks([1.0 + rank, 10.0 - rank], world, dev)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"launcher_check": True, "n_gpus": world, "backend": backend,
+                          "max_over_ranks": got}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200000)
-    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=2, choices=sorted(WORKLOADS))
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--replicas", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config entries of the default line")
+    ap.add_argument("--per-config", action="store_true",
+                    help="add per_config entries to a non-default line")
     ap.add_argument("--shared", action="store_true",
                     help="shared GQA selection (one top-k per kv head)")
     ap.add_argument("--thresholds", default="fixed", choices=["fixed", "absmax"],
@@ -623,22 +730,44 @@ def main():
                     help="time one rank of a W-way context-parallel step (its L/W slice)")
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE",
                     help="hold the caches in a pool of PAGE-token pages (block tables)")
+    ap.add_argument("--policy", default="auto", choices=["auto", "cluster", "flat"],
+                    help="decode kernel: the planner's choice, thread-block clusters only, "
+                         "or the grid-wide kernel wherever it applies")
+    ap.add_argument("--launcher-check", action="store_true",
+                    help="only set up the ranks and reduce over them (no kernels)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    args.steps = max(1, args.steps)
     if args.budget is None:
         args.budget = 128 if 128 in WORKLOADS[args.config].budgets else WORKLOADS[args.config].budgets[0]
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(spawn_ranks(args.gpus))
     rank, world, local = dist_env()
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch with "
+              f"torch.distributed.run --nproc-per-node {args.gpus}, or omit WORLD_SIZE",
+              file=sys.stderr)
+        sys.exit(2)
+    if args.launcher_check:
+        launcher_check(world, local, rank)
+        return
 
     if args.impl == "reference":
+        # the oracle on rank 0's host cores; other ranks have nothing to run
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
 
+    import token_level_sparse_fwht_b200 as ad
+    ad.set_decode_policy({"auto": ad.POLICY_AUTO, "cluster": ad.POLICY_CLUSTER,
+                          "flat": ad.POLICY_FLAT}[args.policy])
     if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    r = run_ours(args, rank, world, local)
+        init_ranks(world, local)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    default_line = (args.config == 2 and args.budget == 128 and not args.shared
+                    and not args.paged and not args.cp and args.thresholds == "fixed")
+    r = measure(args, args.config, args.budget, dev, world)
     w, k = r["w"], r["k"]
     peak, peak_kind = peaks()
     per_step_s = r["ms"] / 1e3 / r["K"]
@@ -658,8 +787,7 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": round(r["ms"] / r["K"], 6),
         "us_per_step": round(per_step_s * 1e6, 3),
-        "us_per_step_median_replay": (round(r["us_median"], 3) if r["us_median"] is not None
-                                      else None),
+        "us_per_step_median_replay": round(r["us_median"], 3),
         "pct_of_roofline": round(100 * gbs_rank / peak, 2),
         "higher_is_better": True,
         "scaling": "weak",
@@ -677,20 +805,35 @@ def main():
                    "replicas": r["R"], "l2": "rotated replicas, working set >= 2x L2",
                    "layers": w.layers, "append_tokens": w.append,
                    "graph": r["use_graph"], "ctas": r["plan"]["ctas"],
+                   "kernel": r["kernel"], "policy": args.policy,
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(gbs_rank / peak, 4),
                      "traffic": ncu_traffic(key),
-                     "kernel": "decode_kernel (one launch per step)",
+                     "kernel": f"{r['kernel']} (one launch per step)",
                      "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": {"value": round(aggregate_gbs(r["step_bytes"], e2e_step_s, world), 2), "unit": "GB/s",
                 "us_per_step": round(e2e_step_s * 1e6, 3),
+                "sync_us_per_step": round(r["sync_us"], 2),
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
     if r["recall"] is not None:
         line["recall_planted_keys"] = r["recall"]
+    if (default_line and not args.no_per_config) or args.per_config:
+        entries = []
+        for cfg, kk in PER_CONFIG:
+            if cfg == args.config and kk == args.budget and default_line:
+                entries.append(per_config_entry(r, peak))
+                continue
+            rr = measure(args, cfg, kk, dev, world, per_config=True)
+            entries.append(per_config_entry(rr, peak))
+            if rr["append_check"] is not None and rank == 0 and world == 1 \
+                    and not args.no_cpu_baseline:
+                entries[-1]["cpu_baseline_append"] = cpu_append_baseline(rr["w"],
+                                                                         *rr["append_check"])
+        line["per_config"] = entries
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, k, shared=args.shared,
                                             absmax=args.thresholds == "absmax")

@@ -76,6 +76,18 @@ const char* adamas_status_string(adamas_status s);
 int adamas_abi_version(void);
 
 /*
+ * Which kernel the decode and select entry points may plan with (process-wide, for
+ * tuning and testing; results are the same either way): 0 = whichever the launch
+ * planner models as faster (the default), 1 = thread-block clusters only (one
+ * cluster per (batch, kv head) unit, exchange in distributed shared memory), 2 =
+ * the grid-wide kernel wherever it applies (contiguous caches with per-query-head
+ * selection and few enough units that every unit gets at least two CTAs, all CTAs
+ * co-resident at one per SM; exchange through the workspace).  Changing it changes
+ * adamas_decode_workspace_bytes for some sizes.  ADAMAS_ERR_INVALID_ARG outside 0..2.
+ */
+adamas_status adamas_set_decode_policy(int policy);
+
+/*
  * Key encoder, run when keys are appended to the cache (v2 abstract: Hadamard
  * transform, bucketization, 2-bit compression of the keys).  Encodes positions
  * [pos0, pos0 + n_new) of every (batch, kv head) from k_cache into codes.

@@ -28,3 +28,14 @@ def read_golden(name):
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+@pytest.fixture(params=[1, 2], ids=["cluster", "flat"])
+def decode_policy(request):
+    """Runs a GPU test once per decode kernel: thread-block clusters, then the
+    grid-wide kernel wherever it applies (sizes it does not cover fall back to
+    clusters).  The planner's default choice is one of the two."""
+    import token_level_sparse_fwht_b200 as ad
+    ad.set_decode_policy(request.param)
+    yield request.param
+    ad.set_decode_policy(0)

@@ -18,7 +18,7 @@ def test_library_exports_every_header_symbol():
     assert "adamas_decode_step" in syms and "adamas_encode_keys" in syms
     for s in syms:
         assert hasattr(lib, s), s
-    assert lib.adamas_abi_version() == 1
+    assert lib.adamas_abi_version() == 2
 
 
 def test_status_strings():
@@ -97,18 +97,41 @@ def test_workspace_sizes_and_plan():
     assert ad.lib().adamas_decode_workspace_bytes(1, 32, 8, 128, 0, 128) == 0
     assert ad.lib().adamas_sparse_attention_workspace_bytes(1, 32, 128) > 0
     assert ad.lib().adamas_sparse_attention_workspace_bytes(1, 32, 0) == 0
-    # without a device the plan assumes a 148-SM B200 and its shared-memory cap
-    p = ad.decode_plan(1, 32, 8, 32768, 128)           # 8 units: clusters of 16
-    assert p == {"ctas": 128, "cluster": 16, "tokens_per_cta": 2048,
+    # without a device the plan assumes a 148-SM B200 (its shared-memory cap and the
+    # cluster occupancy it reports).  The 32K layer's 8 units: clusters of 10 (at most
+    # 11 fit at once); the grid-wide kernel (18 CTAs of 1824 keys per unit) only on
+    # request.  One kv head over 256K: the grid-wide kernel by default.
+    p = ad.decode_plan(1, 32, 8, 32768, 128)
+    assert p == {"ctas": 80, "cluster": 10, "tokens_per_cta": 3277,
                  "smem_bytes": p["smem_bytes"]} and p["smem_bytes"] <= 232448
+    assert ad.decode_workspace_bytes(1, 32, 8, 32768, 128) == 256
+    ad.set_decode_policy(ad.POLICY_FLAT)
+    try:
+        pf = ad.decode_plan(1, 32, 8, 32768, 128)
+        assert pf == {"ctas": 144, "cluster": 1, "tokens_per_cta": 1824,
+                      "smem_bytes": pf["smem_bytes"]}
+        assert ad.decode_workspace_bytes(1, 32, 8, 32768, 128) > 256   # exchange scratch
+    finally:
+        ad.set_decode_policy(ad.POLICY_AUTO)
+    long1 = ad.decode_plan(1, 4, 1, 262144, 128)
+    assert long1["cluster"] == 1 and long1["ctas"] == 64 and long1["tokens_per_cta"] == 4096
+    ad.set_decode_policy(ad.POLICY_CLUSTER)
+    try:
+        assert ad.decode_plan(1, 4, 1, 262144, 128)["cluster"] == 16
+    finally:
+        ad.set_decode_policy(ad.POLICY_AUTO)
+    with pytest.raises(ad.AdamasError):
+        ad.set_decode_policy(3)
     big = ad.decode_plan(8, 32, 8, 32768, 1024)         # 64 units: clusters of 2
     assert big["cluster"] == 2 and big["tokens_per_cta"] == 16384
     for args in [(4, 32, 8, 131072, 1024), (1, 32, 32, 131072, 1024), (1, 2, 1, 70000, 50),
                  (75, 4, 4, 64, 8), (1, 1, 1, 1024, 64)]:
         q = ad.decode_plan(*args)
         B, Hq, Hkv, L, k = args
-        assert q["ctas"] == B * Hkv * q["cluster"] and 1 <= q["cluster"] <= 16
-        assert q["tokens_per_cta"] * q["cluster"] >= L and q["tokens_per_cta"] <= 65535
+        per_unit = q["ctas"] // (B * Hkv)
+        assert q["ctas"] == B * Hkv * per_unit and q["cluster"] in (1, per_unit)
+        assert 1 <= per_unit <= 148 and (q["cluster"] == 1 or q["cluster"] <= 16)
+        assert q["tokens_per_cta"] * per_unit >= L and q["tokens_per_cta"] <= 65535
         assert q["smem_bytes"] <= 232448
     tiny = ad.decode_plan(3, 4, 4, 1, 1)                # L = 1: one key per unit
     assert tiny["cluster"] == 1 and tiny["tokens_per_cta"] == 1 and tiny["ctas"] == 12
@@ -140,7 +163,7 @@ def test_shared_entry_points_reject_and_plan():
         assert q["ctas"] == B * Hkv * q["cluster"] and 1 <= q["cluster"] <= 16
         assert q["tokens_per_cta"] * q["cluster"] >= L and q["tokens_per_cta"] <= 65535
         assert q["smem_bytes"] <= 232448
-    assert ad.decode_plan_shared(1, 32, 8, 32768, 128)["cluster"] == 16
+    assert ad.decode_plan_shared(1, 32, 8, 32768, 128)["cluster"] == 10   # at most 11 fit
 
 
 def test_varlen_and_paged_entry_points_reject():
@@ -241,8 +264,13 @@ def test_context_parallel_entry_points_reject():
 def test_context_parallel_workspace_size():
     # the error word plus, per CTA, its distances (u16 per key and selection head) and
     # cumulative histograms
+    # (a context-parallel slice always runs on thread-block clusters)
     n = ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 128, 16384, 128, 0)
-    p = ad.decode_plan(1, 32, 8, 16384, 128)
+    ad.set_decode_policy(ad.POLICY_CLUSTER)
+    try:
+        p = ad.decode_plan(1, 32, 8, 16384, 128)
+    finally:
+        ad.set_decode_policy(ad.POLICY_AUTO)
     per_cta = 4 * ((p["tokens_per_cta"] + 7) // 8 * 8) * 2 + 4 * 388 * 4
     assert n == 256 + p["ctas"] * per_cta
     assert ad.lib().adamas_cp_workspace_bytes(1, 32, 8, 128, 16384, 128, 2) == 0
@@ -252,9 +280,7 @@ def test_context_parallel_workspace_size():
 def test_scratch_distance_plan_workspace():
     # many units over a long context: the plan keeps each CTA's distances (u16 per key
     # and head) in the workspace, so fewer, longer CTAs run in one wave
-    # (without a device the planner assumes every SM can host a cluster CTA, so it may
-    # keep distances on chip here while the B200 plan uses scratch: check the size
-    # rule whichever plan is chosen)
+    # (check the size rule whichever plan is chosen)
     for B, Hq, Hkv, L, k in [(4, 32, 8, 131072, 1024), (8, 32, 8, 131072, 256),
                              (2, 64, 8, 131072, 512)]:
         p = ad.decode_plan(B, Hq, Hkv, L, k)
@@ -264,4 +290,8 @@ def test_scratch_distance_plan_workspace():
         # a plan without scratch must fit its distances in shared memory
         if n == 256:
             assert (Hq // Hkv) * stride * 2 < p["smem_bytes"]
-    assert ad.decode_workspace_bytes(1, 32, 8, 32768, 128) == 256   # fits on chip
+    ad.set_decode_policy(ad.POLICY_CLUSTER)
+    try:
+        assert ad.decode_workspace_bytes(1, 32, 8, 32768, 128) == 256   # fits on chip
+    finally:
+        ad.set_decode_policy(ad.POLICY_AUTO)

@@ -1,4 +1,5 @@
-"""The fused decode step (one cooperative kernel) vs the float64 oracle.
+"""The fused decode step (one kernel launch: thread-block clusters, or the grid-wide
+kernel for few units; both are run) vs the float64 oracle.
 
 The key codes are the oracle's (uploaded); the kernel encodes the queries itself in
 fp32, so a query coordinate within 1e-4 of a threshold may take either bucket: the
@@ -56,7 +57,7 @@ def _check_all(inp, kc, L, k, heads=None):
     (2, dict(L=777, Hq=4, Hkv=2), 2000),           # k > L: dense
     (2, dict(B=70, Hq=4, Hkv=4, L=64), 5),         # 280 units: two waves
 ])
-def test_decode_step_matches_oracle(cfg, over, k):
+def test_decode_step_matches_oracle(cfg, over, k, decode_policy):
     w = WORKLOADS[cfg].scaled(**over)
     inp = generate(w, "cpu")
     kc = oracle_codes(inp.k_cache, inp.t)
@@ -68,7 +69,7 @@ def test_decode_step_matches_oracle(cfg, over, k):
                 assert set(inp.planted[b, h].tolist()) <= set(idx[b, h].tolist())
 
 
-def test_decode_lmax_padding_and_repeat():
+def test_decode_lmax_padding_and_repeat(decode_policy):
     w = WORKLOADS[2].scaled(L=2000, Hq=8, Hkv=2)
     inp = generate(w, "cpu", Lmax=2600)
     kc = oracle_codes(inp.k_cache, inp.t)
@@ -78,7 +79,7 @@ def test_decode_lmax_padding_and_repeat():
     assert np.array_equal(idx, idx2) and np.array_equal(out, out2)
 
 
-def test_decode_without_idx_output():
+def test_decode_without_idx_output(decode_policy):
     w = WORKLOADS[2].scaled(L=1500, Hq=8, Hkv=2)
     inp = generate(w, "cpu")
     kc = oracle_codes(inp.k_cache, inp.t)
@@ -91,7 +92,7 @@ def test_decode_without_idx_output():
                           f64(inp.v_cache[0, h // 4]), kc[0, h // 4], 64, inp.t)
 
 
-def test_decode_full_32k_layer_every_budget():
+def test_decode_full_32k_layer_every_budget(decode_policy):
     """Llama-3.1-8B-shaped layer, 32K context: all 32 heads at budgets 64..1024, in
     the launch configuration the benchmark times."""
     w = WORKLOADS[2]
@@ -161,7 +162,7 @@ def test_decode_llama8b_128k_layers_sampled():
         torch.cuda.empty_cache()
 
 
-def test_decode_step_host_buffers():
+def test_decode_step_host_buffers(decode_policy):
     """adamas_decode_step_host (pinned q in, fp32 out back, one C call) returns what
     adamas_decode_step returns for the same inputs, bit for bit."""
     w = WORKLOADS[2].scaled(L=2500, Hq=16, Hkv=4)
@@ -180,7 +181,7 @@ def test_decode_step_host_buffers():
     assert torch.equal(out_host, want.cpu())
 
 
-def test_prepared_decode_host_call():
+def test_prepared_decode_host_call(decode_policy):
     """The prepared (buffer-bound) host call gives the same output as decode_step."""
     w = WORKLOADS[2].scaled(L=1800, Hq=8, Hkv=2)
     inp = generate(w, "cpu")
@@ -245,3 +246,19 @@ def test_long_context_plan_with_scratch_distances_decode():
         K, V = f64(inp.k_cache[b, kvh]), f64(inp.v_cache[b, kvh])
         for h in range(kvh * G, (kvh + 1) * G):
             check_decode_head(idx[b, h], out[b, h], q[b, h], K, V, kcs[(b, kvh)], 1024, inp.t)
+
+
+def test_decode_long_single_kv_head_grid_wide_plan():
+    """One kv head over 256K keys (4 query heads): the planner's default is the
+    grid-wide kernel (64 CTAs exchanging counts through the workspace).  Selection on
+    the oracle's codes must be bit-exact and the outputs within 2e-3 for every head."""
+    w = WORKLOADS[2].scaled(Hq=4, Hkv=1, L=262144)
+    plan = ad.decode_plan(1, 4, 1, w.L, 128)
+    assert plan["cluster"] == 1 and plan["ctas"] > 16
+    inp = generate(w, "cuda")
+    kc = oracle_codes(inp.k_cache[0, 0].cpu(), inp.t)[None, None]
+    worst, idx, out, ws = _check_all(type(inp)(q=inp.q.cpu(), k_cache=inp.k_cache.cpu(),
+                                               v_cache=inp.v_cache.cpu(), t=inp.t,
+                                               outlier_channels=None), kc, w.L, 128)
+    assert worst <= 2e-3
+    assert ws.numel() > 256

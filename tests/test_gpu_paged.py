@@ -135,7 +135,7 @@ def _run_decode(inp, kc, lens, k, page, shared, paged=True):
     (1, dict(B=2, L=1024), [1024, 500], 32, 64),                 # fp32, single head
     (2, dict(B=4, L=600, Hq=8, Hkv=4), [600, 5, 599, 300], 8, 1000),  # budget > lengths
 ])
-def test_decode_varlen_matches_oracle(cfg, over, lens, page, k, shared, paged):
+def test_decode_varlen_matches_oracle(cfg, over, lens, page, k, shared, paged, decode_policy):
     w = WORKLOADS[cfg].scaled(**over)
     inp = generate(w, "cpu")
     kc = oracle_codes(inp.k_cache, inp.t)

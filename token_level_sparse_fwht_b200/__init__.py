@@ -39,6 +39,7 @@ _c_p = ctypes.c_void_p
 _SIGNATURES = {
     "adamas_status_string": (ctypes.c_char_p, [_c_i]),
     "adamas_abi_version": (_c_i, []),
+    "adamas_set_decode_policy": (_c_i, [_c_i]),
     "adamas_encode_keys": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i64, _c_f,
                                   _c_p, _c_p]),
     "adamas_encode_queries": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p]),
@@ -122,6 +123,16 @@ def header_symbols():
     with open(HEADER_PATH) as f:
         text = f.read()
     return sorted(set(re.findall(r"\b(adamas_[a-z_0-9]+)\s*\(", text)))
+
+
+POLICY_AUTO, POLICY_CLUSTER, POLICY_FLAT = 0, 1, 2
+
+
+def set_decode_policy(policy: int):
+    """Which decode kernel the planner may use (adamas_set_decode_policy): POLICY_AUTO,
+    POLICY_CLUSTER (thread-block clusters only) or POLICY_FLAT (the grid-wide kernel
+    wherever it applies).  Process-wide; results are the same either way."""
+    _check(lib().adamas_set_decode_policy(int(policy)), "adamas_set_decode_policy")
 
 
 def status_string(s: int) -> str:

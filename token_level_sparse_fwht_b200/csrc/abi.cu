@@ -134,7 +134,13 @@ const char* adamas_status_string(adamas_status s) {
   return "unknown status";
 }
 
-int adamas_abi_version(void) { return 1; }
+int adamas_abi_version(void) { return 2; }
+
+adamas_status adamas_set_decode_policy(int policy) {
+  if (policy < 0 || policy > 2) return ADAMAS_ERR_INVALID_ARG;
+  set_decode_policy(policy);
+  return ADAMAS_OK;
+}
 
 
 
@@ -221,7 +227,7 @@ adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream
   if (cudaMemcpyAsync(&word, p, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return ADAMAS_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ADAMAS_ERR_CUDA;
-  if (word & kErrCopy) return ADAMAS_ERR_TIMEOUT;
+  if (word & (kErrWait | kErrCopy)) return ADAMAS_ERR_TIMEOUT;
   if (word & kErrInput) return ADAMAS_ERR_INVALID_ARG;
   return word ? ADAMAS_ERR_INTERNAL : ADAMAS_OK;
 }

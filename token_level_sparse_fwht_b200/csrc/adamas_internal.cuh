@@ -16,7 +16,8 @@ constexpr int kBinStride = 388;         // padded histogram row
 constexpr int kPartStride = 132;        // m, l, 2 pad, acc[128] (floats)
 
 // error word bits (workspace header)
-constexpr uint32_t kErrCopy = 2u;     // a bounded wait for a copy or a peer gave up
+constexpr uint32_t kErrWait = 1u;     // a bounded wait for peer CTAs gave up
+constexpr uint32_t kErrCopy = 2u;     // a bounded wait for a copy into shared memory gave up
 constexpr uint32_t kErrSelect = 4u;   // top-k bookkeeping found no k-th distance
 constexpr uint32_t kErrInput = 8u;    // a device-resident length or page id out of range
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
@@ -287,6 +288,63 @@ __device__ __forceinline__ uint32_t pair_dist(const PairWords& k, const PairWord
   return r;
 }
 
+// ------------------------------------------------------ decode block shape
+constexpr int kThreads = 512;              // threads per decode CTA
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = kThreads;           // keys per bulk copy (16 KiB of codes), one per thread
+
+// Row stride (u16 elements) of a CTA's per-head distance array: a multiple of 8, so
+// rows start on 16-byte boundaries.
+__host__ __device__ inline int dist_stride(int R) { return (R + 7) & ~7; }
+
+// Bit 15 and bit 31 of w0, then of w1, as bits 0..3 (the sign bits of four packed
+// 16-bit lanes): a byte permute gathers the four high bytes, one multiply moves
+// their top bits to bits 28..31 without carries.
+__device__ __forceinline__ uint32_t lane_sign_bits(uint32_t w0, uint32_t w1) {
+  const uint32_t b = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+  return (b * 0x00204081u) >> 28;
+}
+
+// Exclusive prefix over the block (thread order) of G counters per thread, and the
+// block totals, with one barrier: warp totals go to shared memory, then in every warp
+// lanes 0..kWarps-1 take one total each and a shuffle scan over them gives each
+// warp its offset and the block total.  `scan` holds two buffers of kWarps x G
+// words used alternately (by `parity`), so a call never overwrites totals that a
+// slower warp may still be reading from the previous call.
+template <int G>
+__device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t (&total)[G],
+                                                     uint32_t* scan, int parity, int lane,
+                                                     int warp) {
+  static_assert(kWarps <= 32, "one warp total per lane");
+  uint32_t* buf = scan + parity * kWarps * G;
+  uint32_t inc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    uint32_t x = v[g];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    inc[g] = x;
+    if (lane == 31) buf[warp * G + g] = x;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    uint32_t x = lane < kWarps ? buf[lane * G + g] : 0u;
+#pragma unroll
+    for (int o = 1; o < kWarps; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    // x: inclusive prefix of the warp totals (lane w: warps 0..w)
+    const uint32_t upto = __shfl_sync(0xffffffffu, x, (warp + 31) & 31);
+    total[g] = __shfl_sync(0xffffffffu, x, kWarps - 1);
+    v[g] = (warp > 0 ? upto : 0u) + inc[g] - v[g];
+  }
+}
+
 // ---------------------------------------------------------- warp utilities
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -472,7 +530,13 @@ struct Plan {
   size_t smem;           // dynamic shared memory bytes
   int64_t l2_bytes;      // device L2 capacity (0: unknown)
   bool dist_global;      // distances in workspace scratch, not shared memory
+  bool flat;             // grid-wide kernel: `cluster` = 1, exchange through the workspace
+  int cand_cap;          // flat: candidate slots per head per CTA
 };
+// Which decode kernel the planner may choose: 0 = the faster by its cost model,
+// 1 = thread-block clusters only, 2 = the grid-wide kernel wherever it applies.
+void set_decode_policy(int policy);
+int decode_policy();
 // page_shift: log2(page size) for paged caches, -1 for contiguous caches.  allow_gd:
 // the plan may keep distances in workspace scratch (contiguous per-head kernels).
 bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bool shared,
@@ -513,6 +577,14 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
                           const CpArgs* cpa = nullptr);
 // Distance bins of a selection row: 385 per query head, 384 G + 1 for shared selection.
 inline int selection_bins(int G, bool shared) { return shared ? 384 * G + 1 : 3 * kD + 1; }
+// Grid-wide decode step (contiguous caches, per-query-head selection): plan and launch.
+bool make_flat_plan(int B, int Hq, int Hkv, int64_t L, int k, int sms, int smem_cap, Plan& p);
+size_t flat_workspace_bytes(int B, int Hq, int Hkv, const Plan& p);
+cudaError_t launch_decode_flat(const void* q, const uint8_t* qcodes, const void* k,
+                               const void* v, const uint8_t* codes, adamas_dtype dt, int B,
+                               int Hq, int Hkv, const CacheLayout& lay, int64_t L, int kk,
+                               float t, float t_ratio, void* ws, int32_t* idx_out, float* out,
+                               const Plan& p, cudaStream_t stream);
 cudaError_t launch_cp_combine(const float* partials, int world, int64_t rows, float* out,
                               cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, int64_t nvec,

@@ -27,6 +27,7 @@
 // shared memory of cluster rank 0; after a second cluster barrier rank 0 merges
 // the CS partials and writes the output.
 #include <algorithm>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -40,9 +41,6 @@ namespace cg = cooperative_groups;
 
 namespace adamas {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kChunk = kThreads;  // keys per bulk copy (16 KiB of codes), one per thread
 constexpr int kMaxStages = 8;    // bulk-copy ring depth (runtime: 1..8, as shared memory allows)
 constexpr int kMaxCluster = 16;  // non-portable cluster size limit
 // kernel flavours: contiguous caches, paged caches, one rank of a context-parallel step,
@@ -52,8 +50,6 @@ constexpr int kModeContiguous = 0, kModePaged = 1, kModeCP = 2, kModeContigGD = 
 constexpr int kNCoarse = 30;     // coarse chunks of the D* search (30 x chunk >= bins)
 constexpr int kCoarseRow = 32;   // coarse counts per (CTA, head), padded to 128 B
 constexpr int kRound = kThreads * 32;   // tokens per select round (32 per thread)
-
-__host__ __device__ inline int dist_stride(int R) { return (R + 7) & ~7; }
 
 struct DecodeArgs {
   const void* q;             // [B][Hq][128] (encode mode) or nullptr
@@ -170,54 +166,6 @@ __host__ __device__ inline size_t cp_scratch_per_cta(int GS, int BS, int R) {
 // Page-table entries a CTA stages: the pages its R positions can span.
 __host__ __device__ inline int ptab_entries(int R, int page_shift, bool paged) {
   return paged ? ((R + (1 << page_shift) - 1) >> page_shift) + 1 : 0;
-}
-
-// Bit 15 and bit 31 of w0, then of w1, as bits 0..3 (the sign bits of four packed
-// 16-bit lanes): a byte permute gathers the four high bytes, one multiply moves
-// their top bits to bits 28..31 without carries.
-__device__ __forceinline__ uint32_t lane_sign_bits(uint32_t w0, uint32_t w1) {
-  const uint32_t b = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
-  return (b * 0x00204081u) >> 28;
-}
-
-// Exclusive prefix over the block (thread order) of G counters per thread, and the
-// block totals, with one barrier: warp totals go to shared memory, then in every warp
-// lanes 0..kWarps-1 take one total each and a shuffle scan over them gives each
-// warp its offset and the block total.  `scan` holds two buffers of kWarps x G
-// words used alternately (by `parity`), so a call never overwrites totals that a
-// slower warp may still be reading from the previous call.
-template <int G>
-__device__ __forceinline__ void block_exclusive_scan(uint32_t (&v)[G], uint32_t (&total)[G],
-                                                     uint32_t* scan, int parity, int lane,
-                                                     int warp) {
-  static_assert(kWarps <= 32, "one warp total per lane");
-  uint32_t* buf = scan + parity * kWarps * G;
-  uint32_t inc[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    uint32_t x = v[g];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    inc[g] = x;
-    if (lane == 31) buf[warp * G + g] = x;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    uint32_t x = lane < kWarps ? buf[lane * G + g] : 0u;
-#pragma unroll
-    for (int o = 1; o < kWarps; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    // x: inclusive prefix of the warp totals (lane w: warps 0..w)
-    const uint32_t upto = __shfl_sync(0xffffffffu, x, (warp + 31) & 31);
-    total[g] = __shfl_sync(0xffffffffu, x, kWarps - 1);
-    v[g] = (warp > 0 ? upto : 0u) + inc[g] - v[g];
-  }
 }
 
 template <int G, bool SH, int MD, typename T>
@@ -1131,7 +1079,16 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
       const size_t smem = layout_total(G, shared, int(R), list_cap, cs, stages, ptab, !gd);
       if (smem > size_t(smem_cap)) continue;
       int conc_clusters = sms / cs;
-      if (query_device) conc_clusters = active_clusters(G, shared, cs, smem);
+      if (query_device) {
+        conc_clusters = active_clusters(G, shared, cs, smem);
+      } else if (sms == 148) {
+        // no device to ask: the co-resident clusters of one CTA per SM that
+        // cudaOccupancyMaxActiveClusters reports on a 148-SM B200 (its SMs sit in
+        // GPCs of unequal size, so large clusters fit fewer times than 148 / cs)
+        static const int kB200Clusters[17] = {0, 148, 74, 45, 33, 26, 22, 15, 15, 15, 11,
+                                              7, 7, 7, 7, 7, 7};
+        conc_clusters = kB200Clusters[cs];
+      }
       if (conc_clusters < 1) continue;
       const int64_t total = U * cs;
       const int64_t conc = int64_t(conc_clusters) * cs;
@@ -1150,6 +1107,8 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
         p.waves = int(waves);
         p.l2_bytes = 0;
         p.dist_global = gd != 0;
+        p.flat = false;
+        p.cand_cap = 0;
       }
     }
   }
@@ -1157,17 +1116,50 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int
 }
 
 namespace {
-// Plans are memoised per device and problem: making one queries the cluster
+// Plans are memoised per device, problem and policy: making one queries the cluster
 // occupancy of every candidate cluster size, far more host time than a launch.
 struct PlanKey {
-  int dev, B, Hq, Hkv, k, page_shift;
+  int dev, B, Hq, Hkv, k, page_shift, policy;
   int64_t L;
   bool shared, allow_gd;
   bool operator<(const PlanKey& o) const {
-    return std::tie(dev, B, Hq, Hkv, k, page_shift, L, shared, allow_gd) <
-           std::tie(o.dev, o.B, o.Hq, o.Hkv, o.k, o.page_shift, o.L, o.shared, o.allow_gd);
+    return std::tie(dev, B, Hq, Hkv, k, page_shift, policy, L, shared, allow_gd) <
+           std::tie(o.dev, o.B, o.Hq, o.Hkv, o.k, o.page_shift, o.policy, o.L, o.shared,
+                    o.allow_gd);
   }
 };
+std::atomic<int> g_policy{0};
+
+// Modelled step time of a plan (ns), fitted to B200 measurements of both kernels:
+// waves x (per-key scan cost x keys per CTA + fixed latency of the stage chain).  The
+// cluster kernel's chain (exchanges in distributed shared memory) costs about 8 us.
+// The grid-wide kernel's exchanges are round trips through L2 and its last CTA merges
+// every split, so its chain costs about 14.4 us plus 0.11 us per CTA of a unit: it
+// wins only where clusters would leave most SMs idle over very long contexts (one kv
+// head at 256K: 26.3 against 31.5 us; the 32K Llama layer: 18.7 against 13.0 us).
+double plan_cost(int G, const Plan& p, int64_t units) {
+  const double per_key_ns = (0.477 + 0.243 * G) * (p.dist_global ? 1.15 : 1.0);
+  const double per_unit = units > 0 ? double(p.grid) / double(units) : 1.0;
+  const double fixed = p.flat ? 14400.0 + 110.0 * per_unit : 8000.0;
+  return double(p.waves) * (per_key_ns * double(p.keys_per_cta) + fixed);
+}
+
+// Where it applies (contiguous caches, per-head selection, not a context-parallel
+// slice: callers say so with allow_gd), the grid-wide plan replaces the cluster plan
+// when the policy asks for it or its modelled time is lower.
+void consider_flat(int B, int Hq, int Hkv, int64_t L, int k, bool shared, int page_shift,
+                   bool allow_gd, int sms, int smem_cap, bool have_cluster, Plan& p) {
+  const int policy = g_policy.load();
+  if (policy == 1 || shared || page_shift >= 0 || !allow_gd) return;
+  Plan f;
+  if (!make_flat_plan(B, Hq, Hkv, L, k, sms, smem_cap, f)) return;
+  const int G = Hq / Hkv;
+  const int64_t U = int64_t(B) * Hkv;
+  // by default only where it puts clearly more SMs to work and is modelled faster
+  const bool wider = have_cluster && 4 * int64_t(f.grid) >= 5 * int64_t(p.grid) &&
+                     plan_cost(G, f, U) < plan_cost(G, p, U);
+  if (!have_cluster || policy == 2 || wider) p = f;
+}
 std::mutex g_plan_mutex;
 std::map<PlanKey, std::pair<bool, Plan>> g_plans;
 constexpr size_t kMaxPlans = 4096;
@@ -1179,18 +1171,23 @@ bool decode_plan_for_current_device(int B, int Hq, int Hkv, int64_t L, int k, bo
   const int sms = current_device_sms(&dev);
   if (sms <= 0) {
     // no device visible: plan for a 148-SM part with the sm_100 shared-memory cap
-    return make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, 148, 232448, false,
-                            p);
+    const bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, 148, 232448,
+                                     false, p);
+    consider_flat(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, 148, 232448, ok, p);
+    return ok || p.flat;
   }
-  const PlanKey key{dev, B, Hq, Hkv, k, page_shift, L, shared, allow_gd};
+  const PlanKey key{dev, B, Hq, Hkv, k, page_shift, g_policy.load(), L, shared, allow_gd};
   std::lock_guard<std::mutex> lock(g_plan_mutex);
   const auto it = g_plans.find(key);
   if (it != g_plans.end()) {
     p = it->second.second;
     return it->second.first;
   }
-  const bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, sms,
-                                   max_smem_optin(dev), true, p);
+  p.flat = false;
+  bool ok = make_decode_plan(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, sms,
+                             max_smem_optin(dev), true, p);
+  consider_flat(B, Hq, Hkv, L, k, shared, page_shift, allow_gd, sms, max_smem_optin(dev), ok, p);
+  ok = ok || p.flat;
   int l2 = 0;
   if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
     cudaGetLastError();
@@ -1220,9 +1217,13 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k) {
   if (Hkv <= 0 || Hq % Hkv ||
       !decode_plan_for_current_device(B, Hq, Hkv, L, k, false, -1, p, true))
     return 256;
+  if (p.flat) return flat_workspace_bytes(B, Hq, Hkv, p);
   if (!p.dist_global) return 256;
   return 256 + size_t(p.grid) * (Hq / Hkv) * dist_stride(int(p.keys_per_cta)) * 2;
 }
+
+void set_decode_policy(int policy) { g_policy.store(policy); }
+int decode_policy() { return g_policy.load(); }
 size_t decode_workspace_error_offset() { return 8; }
 
 template <int G, bool SH, int MD, typename T>
@@ -1269,6 +1270,11 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
                           const CacheLayout& lay, int64_t L, int kk, float t, void* ws,
                           int32_t* idx_out, float* out, bool shared, const Plan& p,
                           cudaStream_t stream, float t_ratio, const CpArgs* cpa) {
+  if (p.flat) {
+    if (shared || cpa != nullptr || lay.block_table != nullptr) return cudaErrorInvalidValue;
+    return launch_decode_flat(q, qcodes, k, v, codes, dt, B, Hq, Hkv, lay, L, kk, t, t_ratio, ws,
+                              idx_out, out, p, stream);
+  }
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q; a.qcodes = qcodes; a.k = k; a.v = v; a.codes = codes;

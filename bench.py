@@ -292,77 +292,95 @@ def measure(args, config, k, dev, world, per_config=False):
     stream.synchronize()
     ad.check_workspace(ws, stream)
 
-    # CUDA graphs of `chunk` steps (rotating replicas) + one for the remainder
+    # The K timed steps are captured in CUDA graphs of `chunk` steps (rotating replicas),
+    # the first graph opening with an event-record node and the last closing with one:
+    # the events then bracket exactly the K steps on the device, not the host's
+    # submission of the graph to an idle GPU.  A second set of graphs without event
+    # nodes serves the warm-up and the extra replays behind the median.
     K = args.steps
     chunk = max(1, min(K, 1000 // launches_per_step))
-    graphs = []
+    sizes = [chunk] * (K // chunk) + ([K % chunk] if K % chunk else [])
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    timed, plain = [], []
     use_graph = True
     try:
-        sizes = ([chunk] if K >= chunk else []) + ([K % chunk] if K % chunk else [])
-        for n in sizes:
+        done = 0
+        for gi, n in enumerate(sizes):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.stream(stream):
                 with torch.cuda.graph(g, stream=stream):
+                    if gi == 0:
+                        e0.record(stream)
                     for i in range(n):
-                        step(i, stream)
-            graphs.append((n, g))
+                        step(done + i, stream)
+                    if gi == len(sizes) - 1:
+                        e1.record(stream)
+            timed.append(g)
+            done += n
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(chunk):
+                    step(i, stream)
+        plain.append(g)
     except Exception as e:  # capture unsupported: launch eagerly
         use_graph = False
-        graphs = []
+        timed, plain = [], []
         print(f"# graph capture failed ({e}); eager launches", file=sys.stderr)
     stream.synchronize()
-
-    def replay_k():
-        """Exactly K steps."""
-        if use_graph:
-            for _ in range(K // chunk):
-                graphs[0][1].replay()
-            if K % chunk:
-                graphs[-1][1].replay()
-        else:
-            for i in range(K):
-                step(i, stream)
 
     sampler = ClockSampler(smi_id(dev)) if not per_config else None
     if sampler:
         sampler.start()
-    # W warm-up steps as graph replays, then the timed K steps right behind them (no
-    # idle gap: a GPU left idle drops its clocks)
+    # W warm-up steps (and one untimed run of the timed graphs: a graph's first launch
+    # also uploads it), then the timed K steps
     with torch.cuda.stream(stream):
+        if use_graph:
+            for g in timed:
+                g.replay()
         for _ in range(max(1, math.ceil(args.warmup / max(1, chunk)))):
             if use_graph:
-                graphs[0][1].replay()
+                plain[0].replay()
             else:
                 step(0, stream)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        e0.record(stream)
-        replay_k()
-        e1.record(stream)
+        if use_graph:
+            for g in timed:
+                g.replay()
+        else:
+            e0.record(stream)
+            for i in range(K):
+                step(i, stream)
+            e1.record(stream)
     stream.synchronize()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     ms = e0.elapsed_time(e1)
-    # the median over at least 10 more replays of the K steps (outside the timed region)
+    # median step time over further replays of the timed graphs (at least 10, and for
+    # about 0.6 s, so the clock sampler sees the GPU under this load)
     reps = []
-    with torch.cuda.stream(stream):
-        for _ in range(10 if K * launches_per_step <= 20000 else 3):
-            a_ = torch.cuda.Event(enable_timing=True)
-            b_ = torch.cuda.Event(enable_timing=True)
-            a_.record(stream)
-            replay_k()
-            b_.record(stream)
-            reps.append((a_, b_))
-    stream.synchronize()
-    med_us = statistics.median(a_.elapsed_time(b_) for a_, b_ in reps) * 1e3 / K
+    t_end = time.perf_counter() + (0.6 if sampler else 0.0)
+    while len(reps) < 10 or (time.perf_counter() < t_end and len(reps) < 5000):
+        with torch.cuda.stream(stream):
+            if use_graph:
+                for g in timed:
+                    g.replay()
+            else:
+                e0.record(stream)
+                for i in range(K):
+                    step(i, stream)
+                e1.record(stream)
+        stream.synchronize()
+        reps.append(e0.elapsed_time(e1) * 1e3 / K)
+    med_us = statistics.median(reps)
     clocks = sampler.stop() if sampler else None
     ad.check_workspace(ws, stream)
-    del graphs
+    del timed, plain
 
     # e2e through the public API with host buffers: every step copies its queries in
     # from pinned host memory and reads the fp32 output back
@@ -375,10 +393,20 @@ def measure(args, config, k, dev, world, per_config=False):
     # per layer one C call: pinned q in, fused decode, fp32 out back to pinned host;
     # the calls are bound to their buffers once, as a serving loop would
     calls = None
-    if pc is None and not absmax and not cpW:
-        calls = [[ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws,
-                                        outs[li], out_host[li], stream=stream, shared=shared)
-                  for li, (q, kc, vc, cd) in enumerate(sets[r])] for r in range(R)]
+    if not cpW:
+        def bind(li, kc, vc, cd):
+            if pc is not None:
+                return ad.PreparedPagedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, bt, lens, L,
+                                                  k, t, ws, outs[li], out_host[li], shared=shared,
+                                                  stream=stream)
+            if absmax:
+                return ad.PreparedAbsmaxDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, ratio,
+                                                   ws, outs[li], out_host[li], shared=shared,
+                                                   stream=stream)
+            return ad.PreparedDecodeHost(q_host[li], q_dev[li], kc, vc, cd, L, k, t, ws, outs[li],
+                                         out_host[li], stream=stream, shared=shared)
+        calls = [[bind(li, kc, vc, cd) for li, (q, kc, vc, cd) in enumerate(sets[r])]
+                 for r in range(R)]
 
     def e2e_step(i):
         if cpW:
@@ -386,23 +414,12 @@ def measure(args, config, k, dev, world, per_config=False):
             step(i, stream, q_override=q_dev[0], out_t=outs[0])
             out_host.copy_(outs, non_blocking=True)
             return
-        if calls is None:
-            # paged caches / absmax thresholds: the host copies around the public call
-            q_dev.copy_(q_host, non_blocking=True)
-            for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
-                if pc is None:
-                    ad.decode_step_absmax(q_dev[li], kc, vc, cd, L, k, ratio, ws, shared=shared,
-                                          out=outs[li], stream=stream)
-                    continue
-                if append:
-                    ad.encode_pages(kc, cd, t, page_ids=app_ids, stream=stream)
-                ad.decode_step_paged(q_dev[li], kc, vc, cd, bt, lens, L, k, t, ws, shared=shared,
-                                     out=outs[li], stream=stream)
-            out_host.copy_(outs, non_blocking=True)
-            return
         for li, (q, kc, vc, cd) in enumerate(sets[i % R]):
             if append:
-                ad.encode_keys(kc, cd, L - append, append, t, stream=stream)
+                if pc is not None:
+                    ad.encode_pages(kc, cd, t, page_ids=app_ids, stream=stream)
+                else:
+                    ad.encode_keys(kc, cd, L - append, append, t, stream=stream)
             calls[i % R][li]()
 
     with torch.cuda.stream(stream):

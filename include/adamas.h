@@ -88,6 +88,19 @@ int adamas_abi_version(void);
 adamas_status adamas_set_decode_policy(int policy);
 
 /*
+ * Test hook of the bounded-wait error path (process-wide; not for production use).
+ * While extra_tx_bytes (a multiple of 16, at most 2^20) is nonzero, decode launches
+ * on contiguous caches through thread-block clusters arm the barrier of each CTA's
+ * first code chunk for that many bytes more than the bulk copy delivers, so every
+ * wait on it runs into its 1 s limit.  The kernel then records the timeout in the
+ * workspace error word, stops issuing copies, waits (bounded again) for the copies
+ * it has in flight and returns: adamas_check_workspace reports ADAMAS_ERR_TIMEOUT, the
+ * results of that launch are unspecified, and the device stays usable.  0 restores
+ * normal operation.  ADAMAS_ERR_INVALID_ARG for a negative, unaligned or larger count.
+ */
+adamas_status adamas_test_set_copy_fault(int extra_tx_bytes);
+
+/*
  * Key encoder, run when keys are appended to the cache (v2 abstract: Hadamard
  * transform, bucketization, 2-bit compression of the keys).  Encodes positions
  * [pos0, pos0 + n_new) of every (batch, kv head) from k_cache into codes.
@@ -251,6 +264,26 @@ adamas_status adamas_decode_step_paged(const void* q, const void* k_pages, const
                                        float t, int shared, void* workspace, size_t ws_bytes,
                                        int32_t* idx_out, float* out, cudaStream_t stream);
 
+/*
+ * adamas_decode_step_paged for a caller whose queries and outputs live in host memory
+ * (the serving loop of a paged engine): q_host [B][Hq][d] elements of `dt` in,
+ * out_host [B][Hq][d] float32 back, both asynchronous on `stream` (synchronize
+ * before reading out_host).  Page-locked host buffers mapped into the device's
+ * address space are read and written by the kernel in place (no copies); otherwise
+ * q goes through the caller's device staging buffer q_dev and the output through
+ * out_dev.  Every argument is checked before anything is queued; the rest is as in
+ * adamas_decode_step_paged.
+ */
+adamas_status adamas_decode_step_paged_host(const void* q_host, void* q_dev, const void* k_pages,
+                                            const void* v_pages, const uint8_t* code_pages,
+                                            adamas_dtype dt, int B, int Hq, int Hkv, int d,
+                                            int page_size, int64_t num_pages,
+                                            const int32_t* block_table, int max_blocks_per_seq,
+                                            const int32_t* seq_lens, int64_t max_seq_len, int k,
+                                            float t, int shared, void* workspace,
+                                            size_t ws_bytes, int32_t* idx_out, float* out_dev,
+                                            float* out_host, cudaStream_t stream);
+
 /* Stage entry point: distance scan + top-k over paged codes from query codes. */
 adamas_status adamas_select_topk_paged(const uint8_t* qcodes, const uint8_t* code_pages, int B,
                                        int Hq, int Hkv, int page_size, int64_t num_pages,
@@ -300,6 +333,17 @@ adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, cons
                                         float ratio, int shared, void* workspace,
                                         size_t ws_bytes, int32_t* idx_out, float* out,
                                         cudaStream_t stream);
+
+/* adamas_decode_step_absmax with host-memory queries and outputs: the same buffer
+ * rules as adamas_decode_step_paged_host (mapped page-locked buffers in place, else
+ * copies through q_dev / out_dev; every argument checked before anything is queued). */
+adamas_status adamas_decode_step_absmax_host(const void* q_host, void* q_dev,
+                                             const void* k_cache, const void* v_cache,
+                                             const uint8_t* codes, adamas_dtype dt, int B,
+                                             int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                             int k, float ratio, int shared, void* workspace,
+                                             size_t ws_bytes, int32_t* idx_out, float* out_dev,
+                                             float* out_host, cudaStream_t stream);
 
 /*
  * Context-parallel decode (one GPU per contiguous slice of a long context).  The
@@ -373,9 +417,10 @@ adamas_status adamas_sparse_attention(const void* q, const void* k_cache, const 
  * fixed array inside the library that every GPU loading the library keeps until
  * the process exits.  Limit: B * Hq <= 4096 (larger calls return
  * ADAMAS_ERR_UNSUPPORTED); the split count is reduced so that B * Hq * splits
- * <= 4096.  The FIRST call on each device looks up the array's device address
- * and clears its counters, synchronizing the device; make that first call outside
- * any stream capture.  All calls share the one array (each completed call leaves
+ * <= 4096 (on a 148-SM B200 the default split count never exceeds that).  Every
+ * call looks up the array's device address; the FIRST call on each device (and the
+ * first after a device reset moved the array) clears its counters, synchronizing the
+ * device: make that first call outside any stream capture.  All calls share the one array (each completed call leaves
  * its counters at zero again), so calls that run concurrently on the GPU — from
  * several streams or host threads — race and must be serialized by the caller.
  */

@@ -295,3 +295,12 @@ def test_scratch_distance_plan_workspace():
         assert ad.decode_workspace_bytes(1, 32, 8, 32768, 128) == 256   # fits on chip
     finally:
         ad.set_decode_policy(ad.POLICY_AUTO)
+
+
+def test_copy_fault_hook_rejects_bad_arguments():
+    # the bounded-wait test hook: byte counts must be multiples of 16 in [0, 2^20]
+    # (host-side checks only)
+    assert ad.lib().adamas_test_set_copy_fault(8) == ERR_INVALID_ARG
+    assert ad.lib().adamas_test_set_copy_fault(-16) == ERR_INVALID_ARG
+    assert ad.lib().adamas_test_set_copy_fault((1 << 20) + 16) == ERR_INVALID_ARG
+    assert ad.lib().adamas_test_set_copy_fault(0) == OK

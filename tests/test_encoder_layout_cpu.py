@@ -3,9 +3,14 @@
 The kernel factors the Sylvester H_128 as H_8 (x) H_16 (index i = 16 a + b), multiplies
 each 16-dimension block by H_16 with m16n8k16 MMAs whose k order is permuted (k = 2q,
 2q+1 -> dimensions 4q, 4q+1; k = 2q+8, 2q+9 -> 4q+2, 4q+3), butterflies the 8 blocks,
+buckets each unscaled coordinate y as min(floor(y / tt + 2), 3) (one float32 fused
+multiply-add, a saturating conversion; tt = t sqrt(128); only the sign when t = 0),
 and packs codes from the accumulator layout (row = lane/4 (+8), column = 8 nt + 2
-(lane % 4) + e) through xor-1 and xor-2 lane exchanges.  This emulates those formulas
-lane by lane and compares the bytes with oracle.encode."""
+(lane % 4) + e): lane q puts its nibbles at bits 16 nt + 4 q + 2 e of each block's
+word, the quad ORs the words together (xor-1 and xor-2 exchanges) and lane q stores
+words 2q and 2q + 1.  This emulates those formulas lane by lane and compares the
+bytes with oracle.encode; a code may differ only within float32 rounding of a
+threshold."""
 import numpy as np
 
 import oracle
@@ -26,23 +31,35 @@ def _emulate(X, t):
         for c in range(8):
             if not c & s:
                 z[c], z[c | s] = z[c] + z[c | s], z[c] - z[c | s]
-    tt = t * np.sqrt(128.0)
-    code = lambda y: int(y >= -tt) + int(y >= 0) + int(y >= tt)
+    tt = np.float32(t) * np.float32(np.sqrt(128.0))
+    inv = np.float32(1.0) / tt if tt > 0 else np.float32(np.inf)
+
+    def code(y):
+        if not tt > 0:
+            return 3 if y >= 0 else 0
+        f = np.float32(float(np.float32(y)) * float(inv) + 2.0)   # one rounding, like an fma
+        return int(min(max(np.floor(f), 0.0), 3.0))
+
     out = np.zeros((16, 32), np.uint8)
     for h in range(2):
-        nib = {(ln, a, nt): code(z[a][(ln >> 2) + 8 * h][8 * nt + 2 * (ln & 3)])
-               | (code(z[a][(ln >> 2) + 8 * h][8 * nt + 2 * (ln & 3) + 1]) << 2)
-               for ln in range(32) for a in range(8) for nt in range(2)}
-        byte = {}
-        for (ln, a, nt), mine in nib.items():
-            other = nib[(ln ^ 1, a, nt)]
-            byte[(ln, a, nt)] = (other | (mine << 4)) if ln & 1 else (mine | (other << 4))
-        for ln in range(0, 32, 4):           # lane q = 0 of each quad stores its row
-            words = []
+        part = {}
+        for ln in range(32):
+            q = ln & 3
+            row = (ln >> 2) + 8 * h
             for a in range(8):
-                half = [byte[(ln, a, nt)] | (byte[(ln ^ 2, a, nt)] << 8) for nt in range(2)]
-                words.append(half[0] | (half[1] << 16))
-            out[(ln >> 2) + 8 * h] = np.frombuffer(np.array(words, np.uint32).tobytes(), np.uint8)
+                w = 0
+                for nt in range(2):
+                    c0 = code(z[a][row][8 * nt + 2 * q])
+                    c1 = code(z[a][row][8 * nt + 2 * q + 1])
+                    w |= (c0 | (c1 << 2)) << (16 * nt + 4 * q)
+                part[(ln, a)] = w
+        for ln in range(32):
+            q = ln & 3
+            row = (ln >> 2) + 8 * h
+            full = [part[(ln, a)] | part[(ln ^ 1, a)] | part[(ln ^ 2, a)] | part[(ln ^ 3, a)]
+                    for a in range(8)]
+            words = np.array([full[2 * q], full[2 * q + 1]], np.uint32)
+            out[row, 8 * q:8 * q + 8] = np.frombuffer(words.tobytes(), np.uint8)
     return out
 
 
@@ -56,4 +73,4 @@ def test_mma_encoder_plan_matches_oracle():
         y = oracle.hadamard_rotate(X)
         margin = np.minimum(np.minimum(abs(y + t), abs(y)), abs(y - t))
         diff = oracle.unpack_codes(got) != oracle.unpack_codes(want)
-        assert not (diff & (margin >= 1e-9)).any()
+        assert not (diff & (margin >= 1e-5)).any()

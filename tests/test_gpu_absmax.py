@@ -181,3 +181,29 @@ def test_recall_absmax_vs_fixed_threshold(capsys):
         print(f"\nrecall (needles, dense top-{k}) fixed t: {res['fixed']}, absmax 0.5: "
               f"{res['absmax']}")
     assert res["fixed"][0] >= 0.9 and res["absmax"][0] >= 0.9
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_absmax_host_buffers_match_device_call(pinned):
+    """adamas_decode_step_absmax_host returns what adamas_decode_step_absmax returns,
+    bit for bit, with page-locked (in place) and pageable (staged copies) buffers."""
+    w = WORKLOADS[2].scaled(L=2000, Hq=8, Hkv=2)
+    inp = generate(w, "cpu")
+    kcache, vcache = inp.k_cache.cuda(), inp.v_cache.cuda()
+    codes = upload(oracle.encode_absmax(f64(inp.k_cache), 0.5))
+    ws = ad.decode_workspace(1, 8, 2, w.L, 128)
+    want = ad.decode_step_absmax(inp.q.cuda(), kcache, vcache, codes, w.L, 128, 0.5, ws).cpu()
+    q_host = inp.q.clone()
+    out_host = torch.zeros((1, 8, 128), dtype=torch.float32)
+    if pinned:
+        q_host, out_host = q_host.pin_memory(), out_host.pin_memory()
+    call = ad.PreparedAbsmaxDecodeHost(q_host, torch.empty_like(inp.q, device="cuda"), kcache,
+                                       vcache, codes, w.L, 128, 0.5, ws,
+                                       torch.empty((1, 8, 128), device="cuda"), out_host,
+                                       stream=torch.cuda.current_stream())
+    for _ in range(2):
+        out_host.zero_()
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(out_host, want)
+    ad.check_workspace(ws)

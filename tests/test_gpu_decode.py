@@ -262,3 +262,35 @@ def test_decode_long_single_kv_head_grid_wide_plan():
                                                outlier_channels=None), kc, w.L, 128)
     assert worst <= 2e-3
     assert ws.numel() > 256
+
+
+@pytest.mark.slow
+def test_decode_128k_mha_both_budgets_sampled_heads():
+    """The 128K MHA workload (32 heads, 16 planted needles each) through the fused step
+    at budgets 128 and 1024, in the launch configuration the benchmark times: four
+    sampled heads carry the oracle's key codes (the GPU encoder's elsewhere) and are
+    checked against the oracle in full; the needles are recalled."""
+    w = WORKLOADS[4]
+    inp = generate(w, "cuda")
+    codes = torch.empty(inp.k_cache.shape[:-1] + (32,), dtype=torch.uint8, device="cuda")
+    ad.encode_keys(inp.k_cache, codes, 0, w.L, inp.t)
+    heads = [0, 11, 20, 31]
+    ocodes = {}
+    for h in heads:
+        ocodes[h] = oracle_codes(inp.k_cache[0, h].cpu(), inp.t)
+        codes[0, h] = upload(ocodes[h])
+    q = f64(inp.q)
+    for k in w.budgets:
+        ws = ad.decode_workspace(w.B, w.Hq, w.Hkv, w.L, k)
+        idx = torch.empty((1, w.Hq, k), dtype=torch.int32, device="cuda")
+        out = ad.decode_step(inp.q, inp.k_cache, inp.v_cache, codes, w.L, k, inp.t, ws,
+                             idx_out=idx)
+        torch.cuda.synchronize()
+        ad.check_workspace(ws)
+        gi, go = idx.cpu().numpy(), out.cpu().numpy()
+        for h in heads:
+            err = check_decode_head(gi[0, h], go[0, h], q[0, h], f64(inp.k_cache[0, h]),
+                                    f64(inp.v_cache[0, h]), ocodes[h], k, inp.t)
+            assert err <= 2e-3, (k, h, err)
+        planted = inp.planted[0].cpu().numpy()
+        assert np.mean([np.isin(planted[h], gi[0, h]).mean() for h in range(w.Hq)]) > 0.9

@@ -57,6 +57,22 @@ def test_encode_closed_forms_exact():
     assert got[0, 0] == (3 | 2 << 2 | 2 << 4 | 2 << 6)
 
 
+@pytest.mark.parametrize("t", [0.05, 0.0])
+def test_encode_closed_forms_exact_bf16_tensor_core_path(t):
+    """The same closed forms in bf16 (exact), which go through the tensor-core encoder;
+    t = 0 takes its sign-only bucketing (y = 0 -> code 3)."""
+    x = torch.zeros((1, 1, 130, 128), dtype=torch.bfloat16)
+    x[0, 0, 0] = 1.0
+    for i in range(128):
+        x[0, 0, 1 + i, i] = 1.0
+    x[0, 0, 129] = -1.0
+    codes = torch.zeros((1, 1, 130, 32), dtype=torch.uint8, device="cuda")
+    ad.encode_keys(x.cuda(), codes, 0, 130, t)
+    got = codes.cpu().numpy()[0, 0]
+    want = oracle.encode(x[0, 0].double().numpy(), t)
+    assert np.array_equal(got, want)
+
+
 def test_encode_queries_matches_oracle():
     w = WORKLOADS[2].scaled(B=3)
     inp = generate(w, "cpu")

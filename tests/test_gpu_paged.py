@@ -222,3 +222,35 @@ def test_paged_bad_page_id_and_length_are_reported():
         ad.check_workspace(ws2)
     assert e.value.status == ad.ERR_INVALID_ARG
     assert (idx[1].cpu().numpy() == -1).all()          # length -3 clamped to 0
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_paged_host_buffers_match_device_call(pinned):
+    """adamas_decode_step_paged_host (host q in, host fp32 out, one C call) returns
+    what adamas_decode_step_paged returns, bit for bit: with page-locked buffers the
+    kernel reads and writes them in place; with pageable ones the call copies through
+    the staging buffers."""
+    w = WORKLOADS[2].scaled(B=2, L=1500, Hq=8, Hkv=2)
+    inp = generate(w, "cpu")
+    kc = oracle_codes(inp.k_cache, inp.t)
+    pc = make_block_table([1500, 900], w.L, 16, seed=3)
+    kp = upload(scatter_to_pages(inp.k_cache, pc))
+    vp = upload(scatter_to_pages(inp.v_cache, pc))
+    cp = upload(scatter_to_pages(torch.from_numpy(kc), pc))
+    bt, lens = upload(pc.block_table), upload(pc.seq_lens)
+    ws = ad.decode_workspace(w.B, w.Hq, w.Hkv, w.L, 64)
+    want = ad.decode_step_paged(inp.q.cuda(), kp, vp, cp, bt, lens, w.L, 64, inp.t, ws).cpu()
+    q_host = inp.q.clone()
+    out_host = torch.zeros((w.B, w.Hq, 128), dtype=torch.float32)
+    if pinned:
+        q_host, out_host = q_host.pin_memory(), out_host.pin_memory()
+    call = ad.PreparedPagedDecodeHost(q_host, torch.empty_like(inp.q, device="cuda"), kp, vp, cp,
+                                      bt, lens, w.L, 64, inp.t, ws,
+                                      torch.empty((w.B, w.Hq, 128), device="cuda"), out_host,
+                                      stream=torch.cuda.current_stream())
+    for _ in range(2):
+        out_host.zero_()
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(out_host, want)
+    ad.check_workspace(ws)

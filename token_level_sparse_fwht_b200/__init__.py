@@ -40,6 +40,7 @@ _SIGNATURES = {
     "adamas_status_string": (ctypes.c_char_p, [_c_i]),
     "adamas_abi_version": (_c_i, []),
     "adamas_set_decode_policy": (_c_i, [_c_i]),
+    "adamas_test_set_copy_fault": (_c_i, [_c_i]),
     "adamas_encode_keys": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_i64, _c_i64, _c_f,
                                   _c_p, _c_p]),
     "adamas_encode_queries": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p]),
@@ -76,6 +77,12 @@ _SIGNATURES = {
     "adamas_encode_queries_absmax": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p]),
     "adamas_encode_pages_absmax": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i64, _c_p, _c_i64,
                                           _c_f, _c_p, _c_p]),
+    "adamas_decode_step_paged_host": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i,
+                                             _c_i, _c_i, _c_i64, _c_p, _c_i, _c_p, _c_i64, _c_i,
+                                             _c_f, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p, _c_p]),
+    "adamas_decode_step_absmax_host": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i,
+                                              _c_i, _c_i, _c_i64, _c_i64, _c_i, _c_f, _c_i, _c_p,
+                                              _c_sz, _c_p, _c_p, _c_p, _c_p]),
     "adamas_decode_step_absmax": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i,
                                          _c_i64, _c_i64, _c_i, _c_f, _c_i, _c_p, _c_sz, _c_p,
                                          _c_p, _c_p]),
@@ -133,6 +140,12 @@ def set_decode_policy(policy: int):
     POLICY_CLUSTER (thread-block clusters only) or POLICY_FLAT (the grid-wide kernel
     wherever it applies).  Process-wide; results are the same either way."""
     _check(lib().adamas_set_decode_policy(int(policy)), "adamas_set_decode_policy")
+
+
+def test_set_copy_fault(extra_tx_bytes: int):
+    """adamas_test_set_copy_fault: make the next decode launches' first copy wait run
+    out (test hook of the bounded-wait error path); 0 restores normal operation."""
+    _check(lib().adamas_test_set_copy_fault(int(extra_tx_bytes)), "adamas_test_set_copy_fault")
 
 
 def status_string(s: int) -> str:
@@ -477,6 +490,70 @@ def decode_step_absmax(q, k_cache, v_cache, codes, L: int, k: int, ratio: float,
         _dev(ws, "workspace"), ws.numel(), idx_ptr, _dev(out, "out"), _stream(stream)),
         "adamas_decode_step_absmax")
     return out
+
+
+class _PreparedCall:
+    """One C call bound to fixed buffers (pointers and sizes resolved once)."""
+
+    def __init__(self, name, args, keep):
+        self._name = name
+        self._fn = getattr(lib(), name)
+        self._args = args
+        self._keep = keep
+
+    def __call__(self):
+        status = self._fn(*self._args)
+        if status != OK:
+            raise AdamasError(status, self._name)
+
+
+def _host_pair(q_host, out_host, B, Hq, d):
+    if q_host.is_cuda or out_host.is_cuda:
+        raise ValueError("q_host and out_host must be host tensors")
+    if tuple(q_host.shape) != (B, Hq, d) or tuple(out_host.shape) != (B, Hq, d):
+        raise ValueError("q_host / out_host shapes must be [B, Hq, d]")
+
+
+class PreparedPagedDecodeHost(_PreparedCall):
+    """adamas_decode_step_paged_host bound to fixed buffers: host q in, host fp32 out
+    (mapped page-locked buffers in place, else through q_dev / out_dev)."""
+
+    def __init__(self, q_host, q_dev, k_pages, v_pages, code_pages, block_table, seq_lens,
+                 max_seq_len: int, k: int, t: float, ws, out_dev, out_host, shared: bool = False,
+                 idx_out=None, stream=None):
+        B, Hq, d = q_dev.shape
+        P, Hkv, page, _ = k_pages.shape
+        _host_pair(q_host, out_host, B, Hq, d)
+        args = (_c_p(q_host.data_ptr()), _c_p(_dev(q_dev, "q_dev")), _c_p(_dev(k_pages, "k_pages")),
+                _c_p(_dev(v_pages, "v_pages")), _c_p(_dev(code_pages, "code_pages")),
+                _c_i(_dtype_code(k_pages)), _c_i(B), _c_i(Hq), _c_i(Hkv), _c_i(d), _c_i(page),
+                _c_i64(P), _c_p(_i32(block_table, "block_table")), _c_i(block_table.shape[1]),
+                _c_p(_i32(seq_lens, "seq_lens")), _c_i64(max_seq_len), _c_i(k), _c_f(t),
+                _c_i(int(bool(shared))), _c_p(_dev(ws, "workspace")), _c_sz(ws.numel()),
+                _c_p(None if idx_out is None else _dev(idx_out, "idx_out")),
+                _c_p(_dev(out_dev, "out_dev")), _c_p(out_host.data_ptr()), _c_p(_stream(stream)))
+        super().__init__("adamas_decode_step_paged_host", args,
+                         (q_host, q_dev, k_pages, v_pages, code_pages, block_table, seq_lens, ws,
+                          out_dev, out_host, idx_out))
+
+
+class PreparedAbsmaxDecodeHost(_PreparedCall):
+    """adamas_decode_step_absmax_host bound to fixed buffers."""
+
+    def __init__(self, q_host, q_dev, k_cache, v_cache, codes, L: int, k: int, ratio: float, ws,
+                 out_dev, out_host, shared: bool = False, idx_out=None, stream=None):
+        B, Hq, d = q_dev.shape
+        _, Hkv, Lmax, _ = k_cache.shape
+        _host_pair(q_host, out_host, B, Hq, d)
+        args = (_c_p(q_host.data_ptr()), _c_p(_dev(q_dev, "q_dev")), _c_p(_dev(k_cache, "k_cache")),
+                _c_p(_dev(v_cache, "v_cache")), _c_p(_dev(codes, "codes")),
+                _c_i(_dtype_code(k_cache)), _c_i(B), _c_i(Hq), _c_i(Hkv), _c_i(d), _c_i64(Lmax),
+                _c_i64(L), _c_i(k), _c_f(ratio), _c_i(int(bool(shared))),
+                _c_p(_dev(ws, "workspace")), _c_sz(ws.numel()),
+                _c_p(None if idx_out is None else _dev(idx_out, "idx_out")),
+                _c_p(_dev(out_dev, "out_dev")), _c_p(out_host.data_ptr()), _c_p(_stream(stream)))
+        super().__init__("adamas_decode_step_absmax_host", args,
+                         (q_host, q_dev, k_cache, v_cache, codes, ws, out_dev, out_host, idx_out))
 
 
 # ------------------------------------------------ context-parallel steps

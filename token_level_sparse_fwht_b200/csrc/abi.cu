@@ -136,6 +136,13 @@ const char* adamas_status_string(adamas_status s) {
 
 int adamas_abi_version(void) { return 2; }
 
+adamas_status adamas_test_set_copy_fault(int extra_tx_bytes) {
+  if (extra_tx_bytes < 0 || extra_tx_bytes > (1 << 20) || (extra_tx_bytes % 16))
+    return ADAMAS_ERR_INVALID_ARG;
+  set_copy_fault(uint32_t(extra_tx_bytes));
+  return ADAMAS_OK;
+}
+
 adamas_status adamas_set_decode_policy(int policy) {
   if (policy < 0 || policy > 2) return ADAMAS_ERR_INVALID_ARG;
   set_decode_policy(policy);
@@ -184,30 +191,6 @@ adamas_status adamas_encode_pages_absmax(const void* k_pages, adamas_dtype dt, i
   if (!(ratio > 0.0f)) return ADAMAS_ERR_INVALID_ARG;
   return encode_pages_common(k_pages, dt, Hkv, d, page_size, num_pages, page_ids, n_ids, 0.0f,
                              ratio, code_pages, stream);
-}
-
-adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, const void* v_cache,
-                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
-                                        int Hkv, int d, int64_t Lmax, int64_t L, int k,
-                                        float ratio, int shared, void* workspace,
-                                        size_t ws_bytes, int32_t* idx_out, float* out,
-                                        cudaStream_t stream) {
-  if (!(ratio > 0.0f) || !good_threshold(0.0f, ratio) || (shared != 0 && shared != 1))
-    return ADAMAS_ERR_INVALID_ARG;
-  if (!q || !k_cache || !v_cache || !codes || !workspace || !out) return ADAMAS_ERR_INVALID_ARG;
-  if (!good_dtype(dt)) return ADAMAS_ERR_INVALID_ARG;
-  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
-  if (s != ADAMAS_OK) return s;
-  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(codes, 16) ||
-      !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
-    return ADAMAS_ERR_INVALID_ARG;
-  Plan p;
-  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p, shared == 0))
-    return ADAMAS_ERR_UNSUPPORTED;
-  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
-  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
-                                 contiguous(Lmax), L, k, 0.0f, workspace, idx_out, out,
-                                 shared != 0, p, stream, ratio));
 }
 
 size_t adamas_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t L, int k) {
@@ -360,7 +343,7 @@ adamas_status layout_common(bool shared, const void* q, const uint8_t* qcodes, c
                             const void* vc, const uint8_t* codes, adamas_dtype dt, int B, int Hq,
                             int Hkv, int d, const CacheLayout& lay, int64_t L, int k, float t,
                             void* workspace, size_t ws_bytes, int32_t* idx_out, float* out,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool check_only = false) {
   const bool select_only = q == nullptr;
   if (!codes || !workspace) return ADAMAS_ERR_INVALID_ARG;
   if (select_only ? (!qcodes || !idx_out) : (!kc || !vc || !out)) return ADAMAS_ERR_INVALID_ARG;
@@ -378,8 +361,55 @@ adamas_status layout_common(bool shared, const void* q, const uint8_t* qcodes, c
                                       !shared && page_shift < 0))
     return ADAMAS_ERR_UNSUPPORTED;
   if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  if (check_only) return ADAMAS_OK;
   return from_cuda(launch_decode(q, qcodes, kc, vc, codes, select_only ? ADAMAS_BF16 : dt, B, Hq,
                                  Hkv, lay, L, k, t, workspace, idx_out, out, shared, p, stream));
+}
+
+// Host-buffer form of a decode call whose arguments have been checked: `run(q, out)`
+// launches the device call.  Page-locked host buffers mapped into the device's
+// address space are used in place (the kernel reads q and writes the output through
+// the mapping, no copy-engine work); otherwise q is copied in through q_dev and the
+// output back through out_dev, all asynchronous on `stream`.
+template <typename Run>
+adamas_status with_host_buffers(const void* q_host, void* q_dev, float* out_dev, float* out_host,
+                                size_t qbytes, size_t obytes, cudaStream_t stream, Run run) {
+  const void* qh_dev = mapped_device_pointer(q_host);
+  void* oh_dev = mapped_device_pointer(out_host);
+  if (qh_dev && oh_dev && aligned(qh_dev, 16) && aligned(oh_dev, 16))
+    return run(qh_dev, static_cast<float*>(oh_dev));
+  if (!q_dev || !out_dev || !aligned(q_dev, 16) || !aligned(out_dev, 16))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return ADAMAS_ERR_CUDA;
+  const adamas_status r = run(q_dev, out_dev);
+  if (r != ADAMAS_OK) return r;
+  return from_cuda(cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, stream));
+}
+
+// Per-vector absmax thresholds, contiguous caches (check_only: arguments only).
+adamas_status absmax_common(const void* q, const void* k_cache, const void* v_cache,
+                            const uint8_t* codes, adamas_dtype dt, int B, int Hq, int Hkv, int d,
+                            int64_t Lmax, int64_t L, int k, float ratio, int shared,
+                            void* workspace, size_t ws_bytes, int32_t* idx_out, float* out,
+                            cudaStream_t stream, bool check_only) {
+  if (!(ratio > 0.0f) || !good_threshold(0.0f, ratio) || (shared != 0 && shared != 1))
+    return ADAMAS_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !codes || !workspace || !out) return ADAMAS_ERR_INVALID_ARG;
+  if (!good_dtype(dt)) return ADAMAS_ERR_INVALID_ARG;
+  const adamas_status s = check_decode_sizes(B, Hq, Hkv, d, Lmax, L, k);
+  if (s != ADAMAS_OK) return s;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(codes, 16) ||
+      !aligned(out, 16) || !aligned(workspace, 256) || (idx_out && !aligned(idx_out, 4)))
+    return ADAMAS_ERR_INVALID_ARG;
+  Plan p;
+  if (!decode_plan_for_current_device(B, Hq, Hkv, L, k, shared != 0, -1, p, shared == 0))
+    return ADAMAS_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_workspace_bytes(B, Hq, Hkv, L, k)) return ADAMAS_ERR_INVALID_ARG;
+  if (check_only) return ADAMAS_OK;
+  return from_cuda(launch_decode(q, nullptr, k_cache, v_cache, codes, dt, B, Hq, Hkv,
+                                 contiguous(Lmax), L, k, 0.0f, workspace, idx_out, out,
+                                 shared != 0, p, stream, ratio));
 }
 
 }  // namespace
@@ -473,6 +503,74 @@ adamas_status adamas_decode_step_paged(const void* q, const void* k_pages, const
   if (s != ADAMAS_OK) return s;
   return layout_common(shared != 0, q, nullptr, k_pages, v_pages, code_pages, dt, B, Hq, Hkv, d,
                        lay, max_seq_len, k, t, workspace, ws_bytes, idx_out, out, stream);
+}
+
+adamas_status adamas_decode_step_paged_host(const void* q_host, void* q_dev, const void* k_pages,
+                                            const void* v_pages, const uint8_t* code_pages,
+                                            adamas_dtype dt, int B, int Hq, int Hkv, int d,
+                                            int page_size, int64_t num_pages,
+                                            const int32_t* block_table, int max_blocks_per_seq,
+                                            const int32_t* seq_lens, int64_t max_seq_len, int k,
+                                            float t, int shared, void* workspace,
+                                            size_t ws_bytes, int32_t* idx_out, float* out_dev,
+                                            float* out_host, cudaStream_t stream) {
+  if (!q_host || !out_host || (shared != 0 && shared != 1)) return ADAMAS_ERR_INVALID_ARG;
+  CacheLayout lay;
+  const adamas_status s = check_pages(page_size, num_pages, block_table, max_blocks_per_seq,
+                                      seq_lens, max_seq_len, lay);
+  if (s != ADAMAS_OK) return s;
+  // every argument of the device call is checked before anything is queued (the
+  // aligned workspace pointer stands in for the q / out buffer the mapping decides)
+  void* probe = workspace;
+  const adamas_status c = layout_common(shared != 0, probe, nullptr, k_pages, v_pages, code_pages,
+                                        dt, B, Hq, Hkv, d, lay, max_seq_len, k, t, workspace,
+                                        ws_bytes, idx_out, static_cast<float*>(probe), stream,
+                                        true);
+  if (c != ADAMAS_OK) return c;
+  const size_t qbytes = size_t(B) * Hq * kD * (dt == ADAMAS_F32 ? 4 : 2);
+  const size_t obytes = size_t(B) * Hq * kD * sizeof(float);
+  return with_host_buffers(q_host, q_dev, out_dev, out_host, qbytes, obytes, stream,
+                           [&](const void* qd, float* od) {
+                             return layout_common(shared != 0, qd, nullptr, k_pages, v_pages,
+                                                  code_pages, dt, B, Hq, Hkv, d, lay,
+                                                  max_seq_len, k, t, workspace, ws_bytes,
+                                                  idx_out, od, stream);
+                           });
+}
+
+adamas_status adamas_decode_step_absmax(const void* q, const void* k_cache, const void* v_cache,
+                                        const uint8_t* codes, adamas_dtype dt, int B, int Hq,
+                                        int Hkv, int d, int64_t Lmax, int64_t L, int k,
+                                        float ratio, int shared, void* workspace,
+                                        size_t ws_bytes, int32_t* idx_out, float* out,
+                                        cudaStream_t stream) {
+  return absmax_common(q, k_cache, v_cache, codes, dt, B, Hq, Hkv, d, Lmax, L, k, ratio, shared,
+                       workspace, ws_bytes, idx_out, out, stream, false);
+}
+
+adamas_status adamas_decode_step_absmax_host(const void* q_host, void* q_dev,
+                                             const void* k_cache, const void* v_cache,
+                                             const uint8_t* codes, adamas_dtype dt, int B,
+                                             int Hq, int Hkv, int d, int64_t Lmax, int64_t L,
+                                             int k, float ratio, int shared, void* workspace,
+                                             size_t ws_bytes, int32_t* idx_out, float* out_dev,
+                                             float* out_host, cudaStream_t stream) {
+  if (!q_host || !out_host) return ADAMAS_ERR_INVALID_ARG;
+  // every argument of the device call is checked before anything is queued (the
+  // aligned dummy pointer stands in for the q / out buffer the mapping decides)
+  void* probe = workspace;
+  const adamas_status c = absmax_common(probe, k_cache, v_cache, codes, dt, B, Hq, Hkv, d, Lmax, L,
+                                        k, ratio, shared, workspace, ws_bytes, idx_out,
+                                        static_cast<float*>(probe), stream, true);
+  if (c != ADAMAS_OK) return c;
+  const size_t qbytes = size_t(B) * Hq * kD * (dt == ADAMAS_F32 ? 4 : 2);
+  const size_t obytes = size_t(B) * Hq * kD * sizeof(float);
+  return with_host_buffers(q_host, q_dev, out_dev, out_host, qbytes, obytes, stream,
+                           [&](const void* qd, float* od) {
+                             return absmax_common(qd, k_cache, v_cache, codes, dt, B, Hq, Hkv, d,
+                                                  Lmax, L, k, ratio, shared, workspace, ws_bytes,
+                                                  idx_out, od, stream, false);
+                           });
 }
 
 adamas_status adamas_select_topk_paged(const uint8_t* qcodes, const uint8_t* code_pages, int B,

@@ -533,6 +533,10 @@ struct Plan {
   bool flat;             // grid-wide kernel: `cluster` = 1, exchange through the workspace
   int cand_cap;          // flat: candidate slots per head per CTA
 };
+// Test hook of the copy-wait error path (adamas_test_set_copy_fault): extra bytes the
+// first code chunk's barrier is armed for (the copy never delivers them); 0 restores
+// normal operation.
+void set_copy_fault(uint32_t extra_tx_bytes);
 // Which decode kernel the planner may choose: 0 = the faster by its cost model,
 // 1 = thread-block clusters only, 2 = the grid-wide kernel wherever it applies.
 void set_decode_policy(int policy);

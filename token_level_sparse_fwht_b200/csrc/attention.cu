@@ -5,7 +5,7 @@
 // for sparse attention.  Softmax of (q . K_j) / sqrt(d) over the positions,
 // fp32 accumulation.
 //
-// Grid: (batch x query head) x S splits, 8 warps per CTA, 4 rows in flight per
+// Grid: (batch x query head) x S splits, 8 warps per CTA, 8 rows in flight per
 // warp.  Each CTA writes one softmax partial (m, l, acc[128]); the last CTA of a
 // (batch, head) — atomic counter in the workspace — merges the S partials and
 // resets its counter, so the workspace stays zero between calls.
@@ -140,27 +140,29 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
 static std::mutex g_noalloc_mutex;
-static void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+static void* g_noalloc_cleared[kNoAllocMaxDevices] = {};   // address whose counters were cleared
 
-// Once per device, with that device current: the scratch's device address, and
-// the counters cleared (each completed call returns them to zero by itself).
+// With the calling device current: the scratch's device address, looked up on every
+// call (cheap; a device reset reloads the module and may move the array), and its
+// counters cleared the first time that address is seen (each completed call returns
+// them to zero by itself).
 static cudaError_t noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
+  if (g_noalloc_cleared[dev] != p) {
     e = cudaMemset(p, 0, kNoAllocCounterBytes);
     if (e != cudaSuccess) return e;
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = p;
+    g_noalloc_cleared[dev] = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

@@ -87,6 +87,8 @@ struct DecodeArgs {
   const uint32_t* cp_hist_all;
   int cp_world, cp_rank;
   float* cp_partial;
+  // extra bytes the first chunk's barrier expects (test hook of the copy-wait timeout)
+  uint32_t inject_tx;
 };
 
 // Selection geometry of one kernel flavour.  Per-head selection (SH = false):
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     if constexpr (!paged) {
       const int c0 = qi * kChunk;
       const int keys = min(kChunk, n - c0);
-      mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes));
+      mbar_expect_tx(&mbar[slot], uint32_t(keys * kCodeBytes) + (qi == 0 ? a.inject_tx : 0u));
       bulk_g2s(ring + size_t(slot) * kChunk * kCodeBytes, codes + int64_t(c0) * kCodeBytes,
                uint32_t(keys * kCodeBytes), &mbar[slot]);
     } else {
@@ -278,11 +280,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
   // last warp issues them, so the warps that encode the queries are not delayed.
   // (context-parallel phase 2 reads its distances back from phase 1: no copies)
   const bool scan_codes = !(cp && a.cp_phase == 2);
+  // chunks the issuing thread has put in flight (meaningful in that thread only)
+  int issued = 0;
   if constexpr (!paged) {
     if (tid == kThreads - 32 && scan_codes) {
       for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
       fence_mbar_init();
       for (int qi = 0; qi < min(nch, S); ++qi) issue_chunk(qi, qi);
+      issued = min(nch, S);
     }
   } else {
     // paged: the whole block stages the page table, four independent loads in
@@ -309,6 +314,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
     }
   }
+
+  // A copy wait that gives up sets this thread's copy_abort.  The issuing thread also
+  // scans keys, so it waits on every chunk it issued: once its own wait gave up it
+  // issues no more copies, and before the CTA exits it waits (bounded again) for the
+  // last phase of every slot it filled, so no bulk copy is still writing this CTA's
+  // shared memory when it exits.
+  bool copy_abort = false;
+  const auto drain_copies = [&]() {
+    if constexpr (!paged) {
+      if (tid == kThreads - 32 && copy_abort) {
+        for (int qi = max(0, issued - S); qi < issued; ++qi)
+          mbar_wait_bounded(&mbar[qi % S], uint32_t((qi / S) & 1), a.err);
+      }
+    }
+  };
 
   // ---- prologue: zero histograms, encode (or fetch) the G query codes
   for (int i = tid; i < GS * BS; i += kThreads) hist[i] = 0u;
@@ -449,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           int slot2 = slot + 1;
           uint32_t par2 = parity;
           if (slot2 == S) { slot2 = 0; par2 ^= 1u; }
-          mbar_wait_bounded(&mbar[slot], parity, a.err);
-          mbar_wait_bounded(&mbar[slot2], par2, a.err);
+          if (!mbar_wait_bounded(&mbar[slot], parity, a.err)) copy_abort = true;
+          if (!mbar_wait_bounded(&mbar[slot2], par2, a.err)) copy_abort = true;
           PairWords kt[2];
           load_key(slot, kt[0]);
           load_key(slot2, kt[1]);
@@ -458,9 +478,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           const bool valid[2] = {r[0] < n, r[1] < n};
           score_keys(Two{}, kt, r, valid);
           if (nch > S) __syncthreads();
-          if (tid == kThreads - 32) {
-            if (qi + S < nch) issue_chunk(qi + S, slot);
-            if (qi + 1 + S < nch) issue_chunk(qi + 1 + S, slot2);
+          if (tid == kThreads - 32 && !copy_abort) {
+            if (qi + S < nch) { issue_chunk(qi + S, slot); ++issued; }
+            if (qi + 1 + S < nch) { issue_chunk(qi + 1 + S, slot2); ++issued; }
           }
           slot = slot2 + 1;
           parity = par2;
@@ -473,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         cp_async_wait_pending(S - 1);   // this thread's copies of chunk qi have landed
         __syncwarp();                   // ... and its warp-mates' (the key it scans)
       } else {
-        mbar_wait_bounded(&mbar[slot], parity, a.err);
+        if (!mbar_wait_bounded(&mbar[slot], parity, a.err)) copy_abort = true;
       }
       const int r = qi * kChunk + tid;
       if (r < n) {
@@ -510,7 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         // a slot is refilled only when the CTA's keys need more chunks than the ring
         // holds; otherwise every chunk has its own slot and warps run ahead freely
         if (nch > S) __syncthreads();
-        if (tid == kThreads - 32 && qi + S < nch) issue_chunk(qi + S, slot);
+        if (tid == kThreads - 32 && qi + S < nch && !copy_abort) {
+          issue_chunk(qi + S, slot);
+          ++issued;
+        }
       }
       if (++slot == S) { slot = 0; parity ^= 1u; }
     }
@@ -636,6 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         }
       }
       cluster.sync();
+      drain_copies();
       return;
     }
   }
@@ -970,6 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
           make_float4(A.x * inv, A.y * inv, A.z * inv, A.w * inv);
     }
   }
+  drain_copies();
 }
 
 // ------------------------------------------------------------------- host side
@@ -1129,6 +1154,7 @@ struct PlanKey {
   }
 };
 std::atomic<int> g_policy{0};
+std::atomic<uint32_t> g_inject_tx{0};
 
 // Modelled step time of a plan (ns), fitted to B200 measurements of both kernels:
 // waves x (per-key scan cost x keys per CTA + fixed latency of the stage chain).  The
@@ -1223,6 +1249,7 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int64_t L, int k) {
 }
 
 void set_decode_policy(int policy) { g_policy.store(policy); }
+void set_copy_fault(uint32_t extra_tx_bytes) { g_inject_tx.store(extra_tx_bytes); }
 int decode_policy() { return g_policy.load(); }
 size_t decode_workspace_error_offset() { return 8; }
 
@@ -1302,6 +1329,7 @@ cudaError_t launch_decode(const void* q, const uint8_t* qcodes, const void* k, c
     const int64_t sel_bytes = rows * 2 * kD * (dt == ADAMAS_F32 ? 4 : 2);
     a.prefetch = (p.l2_bytes <= 0 || 4 * sel_bytes <= 3 * p.l2_bytes) ? 1 : 0;
   }
+  a.inject_tx = lay.block_table == nullptr ? g_inject_tx.load() : 0u;
   a.cp_phase = cpa ? cpa->phase : 0;
   a.L_total = cpa ? cpa->L_total : L;
   a.pos_offset = cpa ? cpa->pos_offset : 0;

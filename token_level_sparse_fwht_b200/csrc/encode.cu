@@ -96,11 +96,20 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t code_of(float y, float tt) {
-  return uint32_t(y >= -tt) + uint32_t(y >= 0.0f) + uint32_t(y >= tt);
+// Bucket of an unscaled coordinate y (thresholds at -tt, 0, +tt, tt = t sqrt(128) > 0):
+// floor(y / tt + 2) clamped to [0, 3] — one fused multiply-add and one saturating
+// float -> unsigned conversion (NaN and negatives give 0) plus a min.  It agrees with
+// the three compares except within rounding of a threshold.
+__device__ __forceinline__ uint32_t code_fma(float y, float inv_tt) {
+  return min(__float2uint_rd(fmaf(y, inv_tt, 2.0f)), 3u);
 }
+// t = 0: the thresholds collapse to 0 and only the sign decides (codes 0 and 3).
+__device__ __forceinline__ uint32_t code_sign(float y) { return y >= 0.0f ? 3u : 0u; }
 
-// Same vector and row mapping as encode_rows_kernel; run is a multiple of 16.
+// Same vector and row mapping as encode_rows_kernel; run is a multiple of 16.  A
+// lane's two rows (vectors v + gid and v + gid + 8 of the tile) advance by 16 per
+// tile: their (group, position) pairs are found by one division at the start of the
+// run and then carried forward.
 __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
     const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst, int64_t nvec, int64_t per,
     int64_t stride, int64_t off, int64_t run, float t, const int32_t* __restrict__ ids,
@@ -121,24 +130,35 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
     bfr[nt][1] = h16_pair(4 * q + 2, 4 * q + 3, 8 * nt + gid);
   }
   const float tt = t * 11.313708498984761f;   // sqrt(128)
+  const float inv_tt = 1.0f / tt;             // +inf at t = 0 (the sign path is used)
+  const bool sign_only = !(tt > 0.0f);
+  // nibble (two codes) placement in the 32-bit code word of a 16-dimension block:
+  // output dimension 16 a + 8 nt + 2 q + e sits at bits 16 nt + 4 q + 2 e
+  const uint32_t m0 = 1u << (4 * q), m1 = 1u << (16 + 4 * q);
+  int64_t grp[2], pos[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t vv = v + gid + 8 * h;
+    grp[h] = vv / per;
+    pos[h] = vv - grp[h] * per;
+  }
   for (; v < vend; v += kMmaVecs) {
-    // this lane's two rows: vectors v + gid (h = 0) and v + gid + 8 (h = 1)
     int64_t row[2];
     bool ok[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int64_t vv = v + gid + 8 * h;
-      ok[h] = vv < vend;
-      int64_t g = 0, pos = 0;
-      if (ok[h]) {
-        g = vv / per;
-        pos = vv - g * per;
-        if (ids != nullptr) {
-          g = ids[g];
-          ok[h] = g >= 0 && g < id_limit;
-        }
+      ok[h] = v + gid + 8 * h < vend;
+      int64_t g = grp[h];
+      if (ids != nullptr && ok[h]) {
+        g = ids[g];
+        ok[h] = g >= 0 && g < id_limit;
       }
-      row[h] = g * stride + off + pos;
+      row[h] = g * stride + off + pos[h];
+      pos[h] += kMmaVecs;
+      while (pos[h] >= per) {
+        pos[h] -= per;
+        ++grp[h];
+      }
     }
     uint2 x[2][8];
 #pragma unroll
@@ -175,29 +195,34 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
         }
       }
     }
-    // codes: output dimension 16 a + 8 nt + 2 q + e.  A lane's two coordinates form
-    // half a byte; the xor-1 partner holds the other half, the xor-2 pair the next
-    // byte, so after two shuffles lane q = 0 of each quad has its row's 32 bytes.
+    // codes: each lane fills its nibbles of the 8 code words of each of its two rows,
+    // the quad ORs them together, and lane q stores words 2q and 2q + 1 of each row
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t word[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) {
-        uint32_t half[2];
+        uint32_t nib[2];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const uint32_t nib = code_of(z[a][nt][2 * h], tt) | (code_of(z[a][nt][2 * h + 1], tt) << 2);
-          const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
-          const uint32_t byte = (q & 1) ? (other | (nib << 4)) : (nib | (other << 4));
-          const uint32_t next = __shfl_xor_sync(0xffffffffu, byte, 2);
-          half[nt] = (q & 2) ? (next | (byte << 8)) : (byte | (next << 8));
+          const float y0 = z[a][nt][2 * h], y1 = z[a][nt][2 * h + 1];
+          const uint32_t c0 = sign_only ? code_sign(y0) : code_fma(y0, inv_tt);
+          const uint32_t c1 = sign_only ? code_sign(y1) : code_fma(y1, inv_tt);
+          nib[nt] = c0 + 4u * c1;
         }
-        word[a] = half[0] | (half[1] << 16);
+        uint32_t w = nib[0] * m0 + nib[1] * m1;
+        w |= __shfl_xor_sync(0xffffffffu, w, 1);
+        w |= __shfl_xor_sync(0xffffffffu, w, 2);
+        word[a] = w;
       }
-      if (q == 0 && ok[h]) {
-        uint4* d = reinterpret_cast<uint4*>(dst + row[h] * kCodeBytes);
-        d[0] = make_uint4(word[0], word[1], word[2], word[3]);
-        d[1] = make_uint4(word[4], word[5], word[6], word[7]);
+      if (ok[h]) {
+        uint2* d = reinterpret_cast<uint2*>(dst + row[h] * kCodeBytes) + q;
+        uint32_t lo = word[0], hi = word[1];
+#pragma unroll
+        for (int a = 1; a < 4; ++a) {
+          if (q == a) { lo = word[2 * a]; hi = word[2 * a + 1]; }
+        }
+        *d = make_uint2(lo, hi);
       }
     }
   }

@@ -427,6 +427,132 @@ __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
   }
 }
 
+// attend_rows for bf16 rows with 8 lanes per row: lane l is sub-lane sl = l & 7 of
+// group gq = l >> 3 and holds dimensions 16 sl .. 16 sl + 15 (two 16-byte loads per
+// row of K and of V); the warp's four groups take rows j0 + (4 u + gq) step, so a
+// warp step covers 4 kR rows with three xor-shuffle levels per row instead of five.
+// Each group keeps its own online softmax; at the end the four groups are merged
+// (xor 8, xor 16) and the result is handed over in attend_rows' layout (lane l:
+// dimensions 4 l .. 4 l + 3) in `st`.  qrow: the query, 128 floats (shared memory).
+template <typename PosFn>
+__device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restrict__ kbase,
+                                                    const __nv_bfloat16* __restrict__ vbase,
+                                                    int n, int j0, int step, PosFn pos_of,
+                                                    const float* qrow, float scale_log2,
+                                                    int lane, SoftmaxState& st) {
+  constexpr int kR = 2;   // rows in flight per group
+  const int gq = lane >> 3, sl = lane & 7;
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; i += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(qrow + 16 * sl + i);
+    q[i] = x.x; q[i + 1] = x.y; q[i + 2] = x.z; q[i + 3] = x.w;
+  }
+  float m = -INFINITY, l = 0.f, acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (int jb = j0; jb < n; jb += 4 * kR * step) {
+    uint4 kr[kR][2], vr[kR][2];
+    bool valid[kR];
+#pragma unroll
+    for (int u = 0; u < kR; ++u) {
+      const int jj = jb + (4 * u + gq) * step;
+      valid[u] = jj < n;
+      if (valid[u]) {
+        const int64_t pos = pos_of(jj);
+        const uint4* kp = reinterpret_cast<const uint4*>(kbase + pos * kD) + 2 * sl;
+        const uint4* vp = reinterpret_cast<const uint4*>(vbase + pos * kD) + 2 * sl;
+        kr[u][0] = __ldg(kp);
+        kr[u][1] = __ldg(kp + 1);
+        vr[u][0] = __ldg(vp);
+        vr[u][1] = __ldg(vp + 1);
+      } else {
+        kr[u][0] = kr[u][1] = vr[u][0] = vr[u][1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float s[kR];
+#pragma unroll
+    for (int u = 0; u < kR; ++u) {
+      const uint32_t w[8] = {kr[u][0].x, kr[u][0].y, kr[u][0].z, kr[u][0].w,
+                             kr[u][1].x, kr[u][1].y, kr[u][1].z, kr[u][1].w};
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float lo, hi;
+        bf16x2_to_f32(w[i], lo, hi);
+        d0 = fmaf(q[2 * i], lo, d0);
+        d1 = fmaf(q[2 * i + 1], hi, d1);
+      }
+      s[u] = d0 + d1;
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+#pragma unroll
+      for (int u = 0; u < kR; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+    }
+    float mx = m;
+#pragma unroll
+    for (int u = 0; u < kR; ++u) {
+      s[u] = valid[u] ? s[u] * scale_log2 : -INFINITY;
+      mx = fmaxf(mx, s[u]);
+    }
+    if (mx != -INFINITY) {   // the same in all 8 lanes of a group
+      const float corr = exp2f(m - mx);   // m = -inf -> 0
+      l *= corr;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] *= corr;
+#pragma unroll
+      for (int u = 0; u < kR; ++u) {
+        if (valid[u]) {
+          const float p = exp2f(s[u] - mx);
+          l += p;
+          const uint32_t w[8] = {vr[u][0].x, vr[u][0].y, vr[u][0].z, vr[u][0].w,
+                                 vr[u][1].x, vr[u][1].y, vr[u][1].z, vr[u][1].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float lo, hi;
+            bf16x2_to_f32(w[i], lo, hi);
+            acc[2 * i] = fmaf(p, lo, acc[2 * i]);
+            acc[2 * i + 1] = fmaf(p, hi, acc[2 * i + 1]);
+          }
+        }
+      }
+      m = mx;
+    }
+  }
+  // merge the four groups' states (an empty group has m = -inf, l = 0)
+#pragma unroll
+  for (int o = 8; o < 32; o <<= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+    const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+    const float M = fmaxf(m, mo);
+    const float c1 = M == -INFINITY ? 0.f : exp2f(m - M);
+    const float c2 = M == -INFINITY ? 0.f : exp2f(mo - M);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float ao = __shfl_xor_sync(0xffffffffu, acc[i], o);
+      acc[i] = acc[i] * c1 + ao * c2;
+    }
+    l = l * c1 + lo * c2;
+    m = M;
+  }
+  // hand over: lane L takes dimensions 4 L .. 4 L + 3, held (identically) by every
+  // lane of sub-lane L >> 2; the lane of group L & 3 offers entries 4 (L & 3) + r
+  float mine[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    float v = acc[r];
+#pragma unroll
+    for (int g = 1; g < 4; ++g) v = gq == g ? acc[4 * g + r] : v;
+    mine[r] = v;
+  }
+  const int src = (lane >> 2) + 8 * (lane & 3);
+  st.m = m;
+  st.l = l;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) st.acc[r] = __shfl_sync(0xffffffffu, mine[r], src);
+}
+
 // attend_rows for a group of GM query heads that share one selection: each K/V row
 // is loaded once and scored against all GM queries (q[g][4] is lane's slice of
 // query g); st[g] is head g's state.  kRows rows are in flight per warp.

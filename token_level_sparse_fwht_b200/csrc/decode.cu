@@ -917,7 +917,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       }
     };
     if constexpr (GM == 1) {
-      attend_rows<T>(kb, vb, nsel, sub, WPG, pos_of, qv[0], a.scale_log2, lane, st[0]);
+      // more than 8 rows per warp: bf16 rows go 8 lanes per row (fewer shuffles and
+      // softmax updates per row); otherwise one row per warp instruction, which has
+      // no group merge to pay for
+      bool done = false;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (nsel > 8 * WPG) {
+          attend_rows_bf16_g8(kb, vb, nsel, sub, WPG, pos_of, qf + gi * kD, a.scale_log2, lane,
+                              st[0]);
+          done = true;
+        }
+      }
+      if (!done) attend_rows<T>(kb, vb, nsel, sub, WPG, pos_of, qv[0], a.scale_log2, lane, st[0]);
     } else {
       constexpr int kRowsG = GM <= 2 ? 8 : 4;
       attend_rows_group<T, GM, kRowsG>(kb, vb, nsel, sub, WPG, pos_of, qv, a.scale_log2, lane,

@@ -714,7 +714,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_flat_kernel(const FlatArgs
     SoftmaxState st;
     st.init();
     const auto pos_of = [&](int j) { return int64_t(lrow[j]); };
-    attend_rows<T>(kb, vb, nsel, sub, WPG, pos_of, qv, a.scale_log2, lane, st);
+    // more than 8 rows per warp: bf16 rows go 8 lanes per row
+    bool done = false;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      if (nsel > 8 * WPG) {
+        attend_rows_bf16_g8(kb, vb, nsel, sub, WPG, pos_of, qf + g * kD, a.scale_log2, lane, st);
+        done = true;
+      }
+    }
+    if (!done) attend_rows<T>(kb, vb, nsel, sub, WPG, pos_of, qv, a.scale_log2, lane, st);
     float* mw = merge + (sub * G + g) * kPartStride;
     if (lane == 0) { mw[0] = st.m; mw[1] = st.l; }
 #pragma unroll

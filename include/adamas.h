@@ -120,7 +120,10 @@ adamas_status adamas_encode_queries(const void* q, adamas_dtype dt, int B, int H
 
 /*
  * Workspace of adamas_decode_step and adamas_select_topk, in bytes; 0 if the
- * arguments are invalid or unsupported.  The first 256 bytes hold the device error
+ * arguments are invalid or unsupported.  It serves the selection stage (v2 abstract of
+ * "Adamas: Hadamard Sparse Attention for Efficient Long-Context Inference": the
+ * top-k candidates are the positions whose codes lie closest to the query's code),
+ * which needs, beyond the kernel's own shared memory, only this buffer.  The first 256 bytes hold the device error
  * word that a bounded wait sets when it gives up (see adamas_check_workspace).
  * Where the launch plan keeps every CTA's distances on chip (the 32K layer, for
  * one) that is all of it.  Plans for long contexts over many (batch, kv head) units
@@ -148,7 +151,13 @@ adamas_status adamas_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stre
 adamas_status adamas_check_workspace(const void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
- * One decode step, all five stages in ONE kernel launch (thread-block clusters,
+ * One decode step of the Adamas method (v2 abstract of "Adamas: Hadamard Sparse
+ * Attention for Efficient Long-Context Inference": Hadamard transform, bucketing and
+ * 2-bit compression of the query, a code distance to every cached key (Manhattan, v1
+ * abstract), top-k candidates, and sparse attention over the ORIGINAL K/V rows of
+ * those candidates; the blog "ADAMAS：稀疏注意力优化技术解析与应用实践", section 4,
+ * puts the cost of a 32K decode step in memory traffic), all five stages in ONE
+ * kernel launch (thread-block clusters,
  * one cluster per (batch, kv head) pair, cross-CTA exchange in distributed shared
  * memory): query encode, distance scan over the key codes, exact per-head top-k,
  * gather of the original K/V rows with split softmax attention, and the combine of
@@ -183,7 +192,12 @@ adamas_status adamas_decode_step_host(const void* q_host, void* q_dev, const voi
 
 /*
  * Stage entry point: distance scan + top-k from given query codes (no attention).
- * Same kernel as adamas_decode_step with the attention stages switched off.
+ * Same kernel as adamas_decode_step with the attention stages switched off.  The
+ * stage is the candidate search of the v2 abstract of "Adamas: Hadamard Sparse
+ * Attention for Efficient Long-Context Inference" (smallest code distances to the
+ * query), with the distance the v1 abstract names (Manhattan, summed over the 128
+ * 2-bit codes: 0 .. 384).  qcodes [B][Hq][32] as adamas_encode_queries writes them;
+ * idx_out [B][Hq][k_eff] receives the positions ascending.
  */
 adamas_status adamas_select_topk(const uint8_t* qcodes, const uint8_t* codes, int B, int Hq,
                                  int Hkv, int64_t Lmax, int64_t L, int k, void* workspace,
@@ -399,6 +413,11 @@ size_t adamas_sparse_attention_workspace_bytes(int B, int Hq, int k_eff);
 /*
  * Stage entry point: split-k gather attention + combine over explicit positions
  * idx [B][Hq][k_eff] (any order, each in [0, Lmax)); writes out [B][Hq][d] fp32.
+ * This is the last stage of the v2 abstract of "Adamas: Hadamard Sparse Attention
+ * for Efficient Long-Context Inference": the ORIGINAL K/V states at the selected
+ * positions are gathered and attention runs over them alone, softmax of
+ * (q . K_j) / sqrt(d) with fp32 accumulation.  Positions may repeat; each copy
+ * counts as its own term.  Query head h reads kv head h / G.
  */
 adamas_status adamas_sparse_attention(const void* q, const void* k_cache, const void* v_cache,
                                       adamas_dtype dt, const int32_t* idx, int B, int Hq,

@@ -70,3 +70,17 @@ def test_attention_workspace_reuse():
     b = ad.sparse_attention(inp.q.cuda(), inp.k_cache.cuda(), inp.v_cache.cuda(), idx, ws)
     assert torch.equal(a, b)
     assert int(ws.view(torch.int32)[:8].abs().sum()) == 0
+
+
+def test_attention_repeated_unsorted_positions():
+    """Positions in any order and repeated: each copy is its own softmax term, as in
+    the oracle's K[idx] gather."""
+    w = WORKLOADS[2].scaled(L=700, Hq=8, Hkv=2)
+    inp = generate(w, "cpu")
+    rng = np.random.default_rng(11)
+    idx = rng.integers(0, 40, size=(1, 8, 300)).astype(np.int32)   # many repeats
+    idx[0, 3] = 5                                                  # one row, 300 copies
+    got = ad.sparse_attention(inp.q.cuda(), inp.k_cache.cuda(), inp.v_cache.cuda(),
+                              upload(idx)).cpu().numpy()
+    want = _oracle_attn(f64(inp.q), f64(inp.k_cache), f64(inp.v_cache), idx, w.G)
+    assert np.abs(got - want).max() <= ATOL_OUT

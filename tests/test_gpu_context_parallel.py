@@ -71,7 +71,12 @@ def test_context_parallel_matches_oracle_and_single_gpu(cfg, over, cuts, k, shar
              idx_out=sidx)
     torch.cuda.synchronize()
     assert np.array_equal(idx, sidx.cpu().numpy())
-    assert np.abs(out - sout.cpu().numpy()).max() <= 1e-5
+    # same positions, same float32 arithmetic per row, but the rows' softmax terms are
+    # summed in a different order (ranks first, or the CTAs of one cluster, and within
+    # a warp either one row per instruction or 8-lane row groups merged at the end):
+    # the two agree to float32 rounding of a weighted sum over up to 1024 rows, which
+    # 1e-4 bounds with room (the oracle comparison below keeps 2e-3)
+    assert np.abs(out - sout.cpu().numpy()).max() <= 1e-4
     if not shared:
         q = f64(inp.q)
         G = w.G
@@ -111,7 +116,12 @@ def test_context_parallel_128k_mha_two_ranks_sampled():
                           idx_out=sidx)
     torch.cuda.synchronize()
     assert np.array_equal(idx, sidx.cpu().numpy())
-    assert np.abs(out - sout.cpu().numpy()).max() <= 1e-5
+    # same positions, same float32 arithmetic per row, but the rows' softmax terms are
+    # summed in a different order (ranks first, or the CTAs of one cluster, and within
+    # a warp either one row per instruction or 8-lane row groups merged at the end):
+    # the two agree to float32 rounding of a weighted sum over up to 1024 rows, which
+    # 1e-4 bounds with room (the oracle comparison below keeps 2e-3)
+    assert np.abs(out - sout.cpu().numpy()).max() <= 1e-4
     q = f64(inp.q)
     for h in (0, 7, 19, 31):
         check_decode_head(idx[0, h], out[0, h], q[0, h], f64(inp.k_cache[0, h]),

@@ -434,14 +434,36 @@ __device__ __forceinline__ void attend_rows(const T* __restrict__ kbase,
 // Each group keeps its own online softmax; at the end the four groups are merged
 // (xor 8, xor 16) and the result is handed over in attend_rows' layout (lane l:
 // dimensions 4 l .. 4 l + 3) in `st`.  qrow: the query, 128 floats (shared memory).
+// With `ahead`, the K/V rows of the warp step kAhead steps on are pulled into L2 at
+// every step (lanes 0-3 of each group: one 128-byte line each), so many more rows
+// are on their way from HBM than the registers can hold; callers pass it when the
+// rows were not pulled into L2 earlier.
 template <typename PosFn>
 __device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restrict__ kbase,
                                                     const __nv_bfloat16* __restrict__ vbase,
                                                     int n, int j0, int step, PosFn pos_of,
                                                     const float* qrow, float scale_log2,
-                                                    int lane, SoftmaxState& st) {
-  constexpr int kR = 2;   // rows in flight per group
+                                                    int lane, SoftmaxState& st,
+                                                    bool ahead = false) {
+  constexpr int kR = 2;       // rows in flight per group
+  constexpr int kAhead = 4;   // warp steps between a row's L2 pull and its loads
   const int gq = lane >> 3, sl = lane & 7;
+  const int span = 4 * kR * step;
+  const auto pull = [&](int jb) {
+    if (sl < 4) {
+#pragma unroll
+      for (int u = 0; u < kR; ++u) {
+        const int jj = jb + (4 * u + gq) * step;
+        if (jj < n) {
+          const __nv_bfloat16* row = (sl < 2 ? kbase : vbase) + pos_of(jj) * kD;
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 64 * (sl & 1)));
+        }
+      }
+    }
+  };
+  if (ahead) {
+    for (int d = 0; d < kAhead; ++d) pull(j0 + d * span);
+  }
   float q[16];
 #pragma unroll
   for (int i = 0; i < 16; i += 4) {
@@ -451,7 +473,8 @@ __device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restr
   float m = -INFINITY, l = 0.f, acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int jb = j0; jb < n; jb += 4 * kR * step) {
+  for (int jb = j0; jb < n; jb += span) {
+    if (ahead) pull(jb + kAhead * span);
     uint4 kr[kR][2], vr[kR][2];
     bool valid[kR];
 #pragma unroll

@@ -923,8 +923,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
       bool done = false;
       if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         if (nsel > 8 * WPG) {
+          // rows not pulled into L2 by the select pass are pulled a few steps ahead here
           attend_rows_bf16_g8(kb, vb, nsel, sub, WPG, pos_of, qf + gi * kD, a.scale_log2, lane,
-                              st[0]);
+                              st[0], a.prefetch == 0);
           done = true;
         }
       }

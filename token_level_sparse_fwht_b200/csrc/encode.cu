@@ -106,10 +106,39 @@ __device__ __forceinline__ uint32_t code_fma(float y, float inv_tt) {
 // t = 0: the thresholds collapse to 0 and only the sign decides (codes 0 and 3).
 __device__ __forceinline__ uint32_t code_sign(float y) { return y >= 0.0f ? 3u : 0u; }
 
+// Packed pairs of fp32 values (sm_100 f32x2 arithmetic: one instruction per pair,
+// each lane IEEE round-to-nearest, the same results as two scalar operations).
+__device__ __forceinline__ void add_sub2(float& a0, float& a1, float& b0, float& b1) {
+  // (a, b) <- (a + b, a - b), elementwise on the pairs (a0, a1) and (b0, b1)
+  asm("{\n\t.reg .b64 pa, pb, ps, pd;\n\t"
+      "mov.b64 pa, {%0, %1};\n\t"
+      "mov.b64 pb, {%2, %3};\n\t"
+      "add.rn.f32x2 ps, pa, pb;\n\t"
+      "sub.rn.f32x2 pd, pa, pb;\n\t"
+      "mov.b64 {%0, %1}, ps;\n\t"
+      "mov.b64 {%2, %3}, pd;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+// (y0 m + 2, y1 m + 2) as one packed fused multiply-add
+__device__ __forceinline__ void fma2_plus2(float y0, float y1, float m, float& f0, float& f1) {
+  asm("{\n\t.reg .b64 py, pm, pc, pr;\n\t"
+      "mov.b64 py, {%2, %3};\n\t"
+      "mov.b64 pm, {%4, %4};\n\t"
+      "mov.b64 pc, {%5, %5};\n\t"
+      "fma.rn.f32x2 pr, py, pm, pc;\n\t"
+      "mov.b64 {%0, %1}, pr;\n\t}"
+      : "=f"(f0), "=f"(f1)
+      : "f"(y0), "f"(y1), "f"(m), "f"(2.0f));
+}
+
 // Same vector and row mapping as encode_rows_kernel; run is a multiple of 16.  A
 // lane's two rows (vectors v + gid and v + gid + 8 of the tile) advance by 16 per
 // tile: their (group, position) pairs are found by one division at the start of the
 // run and then carried forward.
+// kSign: t = 0 (codes by sign alone).  Each lane pulls the rows of its next tile into
+// L2 while the current tile is transformed (lane q: line q & 1 of row q >> 1 of its
+// two rows), so the next tile's loads find them there.
+template <bool kSign>
 __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
     const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst, int64_t nvec, int64_t per,
     int64_t stride, int64_t off, int64_t run, float t, const int32_t* __restrict__ ids,
@@ -131,7 +160,6 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
   }
   const float tt = t * 11.313708498984761f;   // sqrt(128)
   const float inv_tt = 1.0f / tt;             // +inf at t = 0 (the sign path is used)
-  const bool sign_only = !(tt > 0.0f);
   // nibble (two codes) placement in the 32-bit code word of a 16-dimension block:
   // output dimension 16 a + 8 nt + 2 q + e sits at bits 16 nt + 4 q + 2 e
   const uint32_t m0 = 1u << (4 * q), m1 = 1u << (16 + 4 * q);
@@ -160,6 +188,15 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
         ++grp[h];
       }
     }
+    {
+      // the next tile's row of this lane's pull (no pull past the run, or through ids)
+      const int h = q >> 1;
+      const int64_t gh = h ? grp[1] : grp[0], ph = h ? pos[1] : pos[0];   // no local array
+      if (ids == nullptr && v + kMmaVecs + gid + 8 * h < vend) {
+        const __nv_bfloat16* nrow = src + (gh * stride + off + ph) * kD;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(nrow + 64 * (q & 1)));
+      }
+    }
     uint2 x[2][8];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -178,7 +215,7 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
                        bfr[nt][1]);
       }
     }
-    // H_8 over the block index
+    // H_8 over the block index, on packed pairs (e, e + 1)
 #pragma unroll
     for (int s = 1; s < 8; s <<= 1) {
 #pragma unroll
@@ -187,11 +224,8 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = z[c][nt][e], p1 = z[c | s][nt][e];
-            z[c][nt][e] = p0 + p1;
-            z[c | s][nt][e] = p0 - p1;
-          }
+          for (int e = 0; e < 4; e += 2)
+            add_sub2(z[c][nt][e], z[c][nt][e + 1], z[c | s][nt][e], z[c | s][nt][e + 1]);
         }
       }
     }
@@ -206,8 +240,16 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const float y0 = z[a][nt][2 * h], y1 = z[a][nt][2 * h + 1];
-          const uint32_t c0 = sign_only ? code_sign(y0) : code_fma(y0, inv_tt);
-          const uint32_t c1 = sign_only ? code_sign(y1) : code_fma(y1, inv_tt);
+          uint32_t c0, c1;
+          if constexpr (kSign) {
+            c0 = code_sign(y0);
+            c1 = code_sign(y1);
+          } else {
+            float f0, f1;
+            fma2_plus2(y0, y1, inv_tt, f0, f1);
+            c0 = min(__float2uint_rd(f0), 3u);
+            c1 = min(__float2uint_rd(f1), 3u);
+          }
           nib[nt] = c0 + 4u * c1;
         }
         uint32_t w = nib[0] * m0 + nib[1] * m1;
@@ -258,7 +300,11 @@ cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, i
     const int64_t mrun = (tiles + mw - 1) / mw * kMmaVecs;
     const int64_t mused = (nvec + mrun - 1) / mrun;
     cfg.gridDim = dim3(static_cast<unsigned>((mused + 7) / 8));
-    return cudaLaunchKernelEx(&cfg, encode_rows_mma_kernel,
+    if (!(t > 0.0f))
+      return cudaLaunchKernelEx(&cfg, encode_rows_mma_kernel<true>,
+                                static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride,
+                                off, mrun, t, ids, id_limit);
+    return cudaLaunchKernelEx(&cfg, encode_rows_mma_kernel<false>,
                               static_cast<const __nv_bfloat16*>(src), dst, nvec, per, stride, off,
                               mrun, t, ids, id_limit);
   }

@@ -142,6 +142,31 @@ __device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) 
   hi = __uint_as_float(w & 0xffff0000u);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction per pair, each
+// element rounded to nearest exactly as the scalar operation would be.
+// (d0, d1) += (a0, a1) * (b0, b1)
+__device__ __forceinline__ void fma_pair(float& d0, float& d1, float a0, float a1, float b0,
+                                         float b1) {
+  asm("{\n\t.reg .b64 pd, pa, pb;\n\t"
+      "mov.b64 pd, {%0, %1};\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 pb, {%4, %5};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pd;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (d0, d1) *= (m, m)
+__device__ __forceinline__ void mul_pair(float& d0, float& d1, float m) {
+  asm("{\n\t.reg .b64 pd, pm;\n\t"
+      "mov.b64 pd, {%0, %1};\n\t"
+      "mov.b64 pm, {%2, %2};\n\t"
+      "mul.rn.f32x2 pd, pd, pm;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(m));
+}
+
 __device__ __forceinline__ void load4(const __nv_bfloat16* row, int lane, float v[4]) {
   const uint2 x = __ldg(reinterpret_cast<const uint2*>(row) + lane);
   bf16x2_to_f32(x.x, v[0], v[1]);
@@ -503,8 +528,7 @@ __device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restr
       for (int i = 0; i < 8; ++i) {
         float lo, hi;
         bf16x2_to_f32(w[i], lo, hi);
-        d0 = fmaf(q[2 * i], lo, d0);
-        d1 = fmaf(q[2 * i + 1], hi, d1);
+        fma_pair(d0, d1, q[2 * i], q[2 * i + 1], lo, hi);
       }
       s[u] = d0 + d1;
     }
@@ -523,7 +547,7 @@ __device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restr
       const float corr = exp2f(m - mx);   // m = -inf -> 0
       l *= corr;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] *= corr;
+      for (int i = 0; i < 16; i += 2) mul_pair(acc[i], acc[i + 1], corr);
 #pragma unroll
       for (int u = 0; u < kR; ++u) {
         if (valid[u]) {
@@ -535,8 +559,7 @@ __device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restr
           for (int i = 0; i < 8; ++i) {
             float lo, hi;
             bf16x2_to_f32(w[i], lo, hi);
-            acc[2 * i] = fmaf(p, lo, acc[2 * i]);
-            acc[2 * i + 1] = fmaf(p, hi, acc[2 * i + 1]);
+            fma_pair(acc[2 * i], acc[2 * i + 1], p, p, lo, hi);
           }
         }
       }

@@ -13,14 +13,17 @@
 // units than fit at once simply run in waves.
 //
 // Exact top-k with ties to the lower position.  Distances are integers 0..384.
-// Each CTA keeps its distances in shared memory and builds, per query head, a
-// 385-bin histogram that it turns into a cumulative one.  After a cluster barrier
-// every CTA reads its peers' cumulative histograms through distributed shared
-// memory — first at 30 coarse bins, then at 14 bins around the crossing — which
-// gives the k-th distance D*, how many tokens of lower-ranked CTAs are selected,
-// and how many of its own D*-ties it takes.  One block scan in position order then
-// emits its selected positions.  The key codes cross HBM exactly once, and no
-// global-memory atomic, barrier or scratch is involved.
+// Each CTA keeps its distances in shared memory (plans for long CTA ranges keep them
+// in workspace scratch, read back from L2) and builds, per query head, a 385-bin
+// histogram that it turns into a cumulative one.  Before a cluster barrier every CTA
+// pushes its cumulative counts at the ends of 30 coarse chunks (13 bins each) into
+// the shared memory of every peer; after it, each CTA finds locally the chunk where
+// the unit's count reaches k, then pulls from each peer a 20-bin window of the
+// cumulative histogram around that chunk through distributed shared memory.  That
+// gives the k-th distance D*, how many tokens of lower-ranked CTAs are selected, and
+// how many of its own D*-ties it takes.  One block scan in position order then emits
+// its selected positions.  The key codes cross HBM exactly once, and no global-memory
+// atomic or barrier is involved.
 //
 // Attention.  Each CTA gathers the original K/V rows it selected (one split of
 // the unit's softmax) and stores its partial (m, l, acc[128]) per head into the

@@ -483,6 +483,42 @@ PER_CONFIG = [(1, 64), (2, 64), (2, 128), (2, 256), (2, 1024), (3, 256), (3, 102
               (4, 1024), (5, 1024)]
 
 
+def measure_encoder(args, dev, world):
+    """Key encode of the workload's whole cache (one layer): adamas_encode_keys over all
+    B x Hkv x L keys, timed alone with CUDA events on the launching stream, the L2
+    flushed (a buffer of 4x L2 written) before every run; median of `--steps` runs
+    after `--warmup`, max over ranks."""
+    import token_level_sparse_fwht_b200 as ad
+    w = WORKLOADS[args.config]
+    inp = generate(w, dev)
+    codes = torch.empty(inp.k_cache.shape[:-1] + (32,), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(4 * l2, dtype=torch.uint8, device=dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xff)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ad.encode_keys(inp.k_cache, codes, 0, w.L, inp.t)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1) * 1e3)
+    us = max_over_ranks([statistics.median(times)], world, dev)[0]
+    nbytes = inp.k_cache.numel() * inp.k_cache.element_size() + codes.numel()
+    peak, peak_kind = peaks()
+    gbs = nbytes / us / 1e3
+    return {"metric": "key encode of the whole cache (one layer), µs and effective HBM GB/s",
+            "value": round(gbs * world, 2), "unit": "GB/s", "n_gpus": world,
+            "us": round(us, 3), "bytes": nbytes, "frac": round(gbs / peak, 4),
+            "peak": peak, "peak_source": f"{peak_kind} hbm_gbs", "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "data": "synthetic",
+            "dtype": str(inp.k_cache.dtype).replace("torch.", ""),
+            "config": {"workload": w.name, "keys": int(inp.k_cache.numel() // 128),
+                       "l2": "flushed before every run"}}
+
+
 def per_config_entry(r, peak):
     w, k = r["w"], r["k"]
     per_step_s = r["ms"] / 1e3 / r["K"]
@@ -752,6 +788,9 @@ def main():
                          "or the grid-wide kernel wherever it applies")
     ap.add_argument("--launcher-check", action="store_true",
                     help="only set up the ranks and reduce over them (no kernels)")
+    ap.add_argument("--encoder", action="store_true",
+                    help="time adamas_encode_keys over the workload's whole key cache "
+                         "(one layer) instead of the decode step")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     args.steps = max(1, args.steps)
@@ -782,6 +821,13 @@ def main():
         init_ranks(world, local)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.encoder:
+        r = measure_encoder(args, dev, world)
+        if rank == 0:
+            print(json.dumps(r), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     default_line = (args.config == 2 and args.budget == 128 and not args.shared
                     and not args.paged and not args.cp and args.thresholds == "fixed")
     r = measure(args, args.config, args.budget, dev, world)

@@ -7,6 +7,8 @@
 // Method: "Adamas: Hadamard Sparse Attention for Efficient Long-Context
 // Inference", v2 abstract (Hadamard transform, bucketization, 2-bit compression)
 // and the blog section 2.2 bucket rule (three thresholds, strict "<").
+#include <mutex>
+
 #include "adamas_internal.cuh"
 
 namespace adamas {
@@ -78,6 +80,13 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ 
 // 4q+2, 4q+3 (q = lane % 4); B = H_16 takes its rows in the same order.  Codes are
 // compared against t sqrt(128) on the unscaled sums.
 constexpr int kMmaVecs = 16;
+// staging: a 256-byte row padded to 288 bytes, so that the 8-byte fragment reads of a
+// warp (rows gid, columns 32 a + 8 q) touch every bank once per 16 lanes
+constexpr int kRowPitch = 288;
+constexpr int kStageBytes = kMmaVecs * kRowPitch;
+constexpr int kEncStages = 2;                            // tiles in flight per warp
+constexpr int kEncSmem = 8 * kEncStages * kStageBytes;   // 8 warps per block
+extern __shared__ __align__(16) uint8_t enc_smem[];
 
 // bf16 bits of H_16[d0][n] (low half) and H_16[d1][n] (high half): +-1.0
 __device__ __forceinline__ uint32_t h16_pair(int d0, int d1, int n) {
@@ -135,9 +144,12 @@ __device__ __forceinline__ void fma2_plus2(float y0, float y1, float m, float& f
 // lane's two rows (vectors v + gid and v + gid + 8 of the tile) advance by 16 per
 // tile: their (group, position) pairs are found by one division at the start of the
 // run and then carried forward.
-// kSign: t = 0 (codes by sign alone).  Each lane pulls the rows of its next tile into
-// L2 while the current tile is transformed (lane q: line q & 1 of row q >> 1 of its
-// two rows), so the next tile's loads find them there.
+// kSign: t = 0 (codes by sign alone).  Tiles are staged in shared memory: each warp
+// keeps kEncStages buffers of 16 rows and copies the tile kEncStages - 1 ahead with
+// 16-byte asynchronous copies (lane (gid, q): chunks q, q + 4, q + 8, q + 12 of its two
+// rows) before it transforms the current one, so HBM reads overlap the arithmetic.
+// Rows whose copy is skipped (past the run, or an invalid page id) leave stale bytes in
+// their buffer rows; the MMA keeps rows apart and their codes are not stored.
 template <bool kSign>
 __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
     const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst, int64_t nvec, int64_t per,
@@ -170,12 +182,13 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
     grp[h] = vv / per;
     pos[h] = vv - grp[h] * per;
   }
-  for (; v < vend; v += kMmaVecs) {
-    int64_t row[2];
-    bool ok[2];
+  // this warp's staging buffers: [kEncStages][16 rows][kRowPitch bytes]
+  uint8_t* const stage = enc_smem + (threadIdx.x >> 5) * kEncStages * kStageBytes;
+  // rows (and validity) of this lane's two vectors in the tile at vt; advances grp, pos
+  const auto tile_rows = [&](int64_t vt, int64_t (&row)[2], bool (&ok)[2]) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      ok[h] = v + gid + 8 * h < vend;
+      ok[h] = vt + gid + 8 * h < vend;
       int64_t g = grp[h];
       if (ids != nullptr && ok[h]) {
         g = ids[g];
@@ -188,22 +201,58 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
         ++grp[h];
       }
     }
-    {
-      // the next tile's row of this lane's pull (no pull past the run, or through ids)
-      const int h = q >> 1;
-      const int64_t gh = h ? grp[1] : grp[0], ph = h ? pos[1] : pos[0];   // no local array
-      if (ids == nullptr && v + kMmaVecs + gid + 8 * h < vend) {
-        const __nv_bfloat16* nrow = src + (gh * stride + off + ph) * kD;
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(nrow + 64 * (q & 1)));
-      }
-    }
-    uint2 x[2][8];
+  };
+  // lane (gid, q) copies 16-byte chunks q, q + 4, q + 8, q + 12 of its two rows
+  const auto copy_tile = [&](int sb, const int64_t (&row)[2], const bool (&ok)[2]) {
+    uint8_t* dstb = stage + sb * kStageBytes;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint2* rp = reinterpret_cast<const uint2*>(src + row[h] * kD) + q;
+      if (ok[h]) {
+        const uint8_t* g = reinterpret_cast<const uint8_t*>(src + row[h] * kD);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) x[h][a] = ok[h] ? __ldg(rp + 4 * a) : make_uint2(0u, 0u);
+        for (int m = 0; m < 4; ++m)
+          cp_async_16(dstb + (gid + 8 * h) * kRowPitch + 16 * (q + 4 * m), g + 16 * (q + 4 * m));
+      }
     }
+    cp_async_commit();
+  };
+  // rows of the tiles in flight: ring[i] belongs to the tile i tiles after this one
+  int64_t row[kEncStages][2];
+  bool ok[kEncStages][2];
+#pragma unroll
+  for (int i = 0; i < kEncStages - 1; ++i) {
+    const int64_t vt = v + i * kMmaVecs;
+    if (vt < vend) {
+      tile_rows(vt, row[i], ok[i]);
+      copy_tile(i, row[i], ok[i]);
+    } else {
+      cp_async_commit();
+    }
+  }
+  for (int sb = 0; v < vend; v += kMmaVecs, sb = sb + 1 == kEncStages ? 0 : sb + 1) {
+    // the copies of the tile kEncStages - 1 ahead go out before this tile is transformed
+    {
+      const int64_t vt = v + (kEncStages - 1) * kMmaVecs;
+      int sn = sb + kEncStages - 1;
+      if (sn >= kEncStages) sn -= kEncStages;
+      if (vt < vend) {
+        tile_rows(vt, row[kEncStages - 1], ok[kEncStages - 1]);
+        copy_tile(sn, row[kEncStages - 1], ok[kEncStages - 1]);
+      } else {
+        cp_async_commit();   // an empty group keeps the wait count uniform
+      }
+    }
+    cp_async_wait_pending(kEncStages - 1);
+    __syncwarp();
+    uint2 x[2][8];
+    const uint8_t* cur = stage + sb * kStageBytes;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+        x[h][a] = *reinterpret_cast<const uint2*>(cur + (gid + 8 * h) * kRowPitch + 32 * a + 8 * q);
+    }
+    __syncwarp();   // every lane has read this buffer before it is refilled
     // z[c][nt][.]: block c times H_16; rows (gid, gid + 8) x columns 8 nt + 2 q + {0, 1}
     float z[8][2][4];
 #pragma unroll
@@ -257,14 +306,22 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
         w |= __shfl_xor_sync(0xffffffffu, w, 2);
         word[a] = w;
       }
-      if (ok[h]) {
-        uint2* d = reinterpret_cast<uint2*>(dst + row[h] * kCodeBytes) + q;
+      if (ok[0][h]) {
+        uint2* d = reinterpret_cast<uint2*>(dst + row[0][h] * kCodeBytes) + q;
         uint32_t lo = word[0], hi = word[1];
 #pragma unroll
         for (int a = 1; a < 4; ++a) {
           if (q == a) { lo = word[2 * a]; hi = word[2 * a + 1]; }
         }
         *d = make_uint2(lo, hi);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i + 1 < kEncStages; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        row[i][h] = row[i + 1][h];
+        ok[i][h] = ok[i + 1][h];
       }
     }
   }
@@ -292,7 +349,18 @@ cudaError_t launch_encode_rows(const void* src, adamas_dtype dt, uint8_t* dst, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (dt == ADAMAS_BF16 && ratio == 0.0f && reinterpret_cast<uintptr_t>(dst) % 16 == 0 &&
-      reinterpret_cast<uintptr_t>(src) % 8 == 0) {
+      reinterpret_cast<uintptr_t>(src) % 16 == 0) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+      attr_err = cudaFuncSetAttribute(encode_rows_mma_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmem);
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(encode_rows_mma_kernel<true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmem);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    cfg.dynamicSmemBytes = kEncSmem;
     // 2 blocks of 8 warps per SM; each warp a run of whole 16-vector tiles
     const int64_t mw_max = int64_t(sms > 0 ? sms : 148) * 16;
     const int64_t tiles = (nvec + kMmaVecs - 1) / kMmaVecs;

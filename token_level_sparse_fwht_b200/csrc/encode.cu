@@ -77,8 +77,10 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const T* __restrict__ 
 // are then butterflied in registers (H_8).  The MMA's k order inside a block is
 // permuted so that a lane's A registers hold 4 consecutive dimensions (one 8-byte
 // load per row and block): k = 2q, 2q+1 -> dimensions 4q, 4q+1 and k = 2q+8, 2q+9 ->
-// 4q+2, 4q+3 (q = lane % 4); B = H_16 takes its rows in the same order.  Codes are
-// compared against t sqrt(128) on the unscaled sums.
+// 4q+2, 4q+3 (q = lane % 4); B = H_16 takes its rows in the same order, and its
+// columns in an order that leaves block coordinates 4q .. 4q+3 in lane q's
+// accumulators (one byte of each code word).  Codes are compared against t sqrt(128)
+// on the unscaled sums.
 constexpr int kMmaVecs = 16;
 // staging: a 256-byte row padded to 288 bytes, so that the 8-byte fragment reads of a
 // warp (rows gid, columns 32 a + 8 q) touch every bank once per 16 lanes
@@ -167,14 +169,17 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
   uint32_t bfr[2][2];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    bfr[nt][0] = h16_pair(4 * q, 4 * q + 1, 8 * nt + gid);
-    bfr[nt][1] = h16_pair(4 * q + 2, 4 * q + 3, 8 * nt + gid);
+    // output column n = gid of tile nt is block coordinate 4 (n >> 1) + 2 nt + (n & 1),
+    // so that lane q ends up holding coordinates 4 q .. 4 q + 3 of every block
+    const int col = 4 * (gid >> 1) + 2 * nt + (gid & 1);
+    bfr[nt][0] = h16_pair(4 * q, 4 * q + 1, col);
+    bfr[nt][1] = h16_pair(4 * q + 2, 4 * q + 3, col);
   }
   const float tt = t * 11.313708498984761f;   // sqrt(128)
   const float inv_tt = 1.0f / tt;             // +inf at t = 0 (the sign path is used)
-  // nibble (two codes) placement in the 32-bit code word of a 16-dimension block:
-  // output dimension 16 a + 8 nt + 2 q + e sits at bits 16 nt + 4 q + 2 e
-  const uint32_t m0 = 1u << (4 * q), m1 = 1u << (16 + 4 * q);
+  // byte-transpose selectors of the quad exchange (partner q ^ 1, then q ^ 2)
+  const uint32_t selA = (q & 1) ? 0x3715u : 0x6240u;
+  const uint32_t selB = (q & 2) ? 0x3276u : 0x5410u;
   int64_t grp[2], pos[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -278,14 +283,15 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
         }
       }
     }
-    // codes: each lane fills its nibbles of the 8 code words of each of its two rows,
-    // the quad ORs them together, and lane q stores words 2q and 2q + 1 of each row
+    // codes: lane q holds coordinates 16 a + 4 q .. 16 a + 4 q + 3 of each row, i.e.
+    // byte q of code word a.  Its bytes of the even and the odd words go into two
+    // registers, a 4 x 4 byte transpose across the lane quad (two exchanges) turns
+    // them into whole words 2 q and 2 q + 1, and lane q stores those.
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t word[8];
+      uint32_t pw[2] = {0u, 0u};   // bytes of words 0, 2, 4, 6 and of words 1, 3, 5, 7
 #pragma unroll
       for (int a = 0; a < 8; ++a) {
-        uint32_t nib[2];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const float y0 = z[a][nt][2 * h], y1 = z[a][nt][2 * h + 1];
@@ -299,21 +305,18 @@ __global__ void __launch_bounds__(256) encode_rows_mma_kernel(
             c0 = min(__float2uint_rd(f0), 3u);
             c1 = min(__float2uint_rd(f1), 3u);
           }
-          nib[nt] = c0 + 4u * c1;
+          const int sh = 8 * (a >> 1) + 4 * nt;   // coordinates 4 q + 2 nt, + 1
+          pw[a & 1] |= (c0 | (c1 << 2)) << sh;
         }
-        uint32_t w = nib[0] * m0 + nib[1] * m1;
-        w |= __shfl_xor_sync(0xffffffffu, w, 1);
-        w |= __shfl_xor_sync(0xffffffffu, w, 2);
-        word[a] = w;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        pw[i] = __byte_perm(pw[i], __shfl_xor_sync(0xffffffffu, pw[i], 1), selA);
+        pw[i] = __byte_perm(pw[i], __shfl_xor_sync(0xffffffffu, pw[i], 2), selB);
       }
       if (ok[0][h]) {
         uint2* d = reinterpret_cast<uint2*>(dst + row[0][h] * kCodeBytes) + q;
-        uint32_t lo = word[0], hi = word[1];
-#pragma unroll
-        for (int a = 1; a < 4; ++a) {
-          if (q == a) { lo = word[2 * a]; hi = word[2 * a + 1]; }
-        }
-        *d = make_uint2(lo, hi);
+        *d = make_uint2(pw[0], pw[1]);
       }
     }
 #pragma unroll

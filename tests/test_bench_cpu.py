@@ -29,3 +29,32 @@ def test_cpu_baseline_samples_layers_and_scales():
     r = bench.cpu_baseline(w, 64, budget_s=0.2, max_threads=1)
     assert "layers [" in r["sample"] and "jobs (scaled)" in r["sample"]
     assert r["value"] > 0
+
+
+def test_traffic_record_follows_the_decode_sources(tmp_path, monkeypatch):
+    """The ncu traffic in the bench line is reported only while the decode kernel's
+    sources (comments and white space aside) are the ones it was captured on."""
+    import json
+    import shutil
+    csrc = tmp_path / "token_level_sparse_fwht_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in bench.DECODE_SOURCES + ("encode.cu",):
+        shutil.copy(os.path.join(bench.ROOT, "token_level_sparse_fwht_b200", "csrc", name),
+                    csrc / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.csrc_digest()
+    rec = tmp_path / "traffic.json"
+    rec.write_text(json.dumps({"cfg": {"csrc_sha": digest, "dram_bytes_per_launch": 123}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    assert bench.ncu_traffic("cfg") == 123
+    assert bench.ncu_traffic("other") is None
+    # an encoder edit or a comment in a decode source leaves the record valid ...
+    (csrc / "encode.cu").write_text("// changed\n")
+    with open(csrc / "decode.cu", "a") as f:
+        f.write("\n// a comment\n")
+    assert bench.csrc_digest() == digest and bench.ncu_traffic("cfg") == 123
+    # ... a code change in one does not
+    with open(csrc / "adamas_internal.cuh", "a") as f:
+        f.write("\nnamespace extra_ns {}\n")
+    assert bench.csrc_digest() != digest and bench.ncu_traffic("cfg") is None
+

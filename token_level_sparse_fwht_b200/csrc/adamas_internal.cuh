@@ -475,7 +475,7 @@ __device__ __forceinline__ void attend_rows_bf16_g8(const __nv_bfloat16* __restr
                                                     int lane, SoftmaxState& st,
                                                     bool ahead = false) {
   constexpr int kR = 2;       // rows in flight per group
-  constexpr int kAhead = 4;   // warp steps between a row's L2 pull and its loads
+  constexpr int kAhead = 2;   // warp steps between a row's L2 pull and its loads
   const int gq = lane >> 3, sl = lane & 7;
   const int span = 4 * kR * step;
   const auto pull = [&](int jb) {
